@@ -1,0 +1,130 @@
+"""Python access to the C oracle (oracle/ll_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and
+the benchmark's CPU-baseline leg are the only callers.  The product path
+never imports this package.
+
+The oracle is the plain binary64 definition of the LiteLinear forward
+(LiteLinear README, introduction, the display formula
+``y = (x B^T) A^T + scale * (x Q_fp8^T) + bias``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+EXACT = 0
+MIRROR = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ll_oracle.c")
+_LIB = os.path.join(_HERE, "libll_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (OpenMP) into oracle/libll_oracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-fno-fast-math", "-ffp-contract=off",
+                               _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        L.llo_dec_e4m3.restype = ctypes.c_double
+        L.llo_dec_e4m3.argtypes = [ctypes.c_uint8]
+        L.llo_dec_bf16.restype = ctypes.c_double
+        L.llo_dec_bf16.argtypes = [ctypes.c_uint16]
+        L.llo_enc_bf16_rne.restype = ctypes.c_uint16
+        L.llo_enc_bf16_rne.argtypes = [ctypes.c_double]
+        L.llo_num_threads.restype = ctypes.c_int
+        p = ctypes.c_void_p
+        L.llo_forward.restype = ctypes.c_int
+        L.llo_forward.argtypes = [ctypes.c_int] * 4 + [p, p, p, p, p, ctypes.c_int, p,
+                                                       ctypes.c_int, p, ctypes.c_int, p]
+        _lib = L
+    return _lib
+
+
+def dec_e4m3(c: int) -> float:
+    return lib().llo_dec_e4m3(int(c))
+
+
+def dec_bf16(b: int) -> float:
+    return lib().llo_dec_bf16(int(b))
+
+
+def enc_bf16_rne(v: float) -> int:
+    return lib().llo_enc_bf16_rne(float(v))
+
+
+def num_threads() -> int:
+    return lib().llo_num_threads()
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def forward(x, B, A, Q, scale, scale_mode, bias=None, mode=EXACT, rows=None):
+    """Reference forward in binary64.
+
+    x: uint16 [M,K] (bf16 bits); B: uint16 [r,K] or None; A: uint16 [N,r]
+    or None; Q: uint8 [N,K] (e4m3fn codes); scale: float32 [N] or [1];
+    bias: uint16 [N] or None.  rows: optional int sequence of row indices
+    of x to evaluate.  Returns float64 [len(rows) or M, N].
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    Q = np.ascontiguousarray(Q, dtype=np.uint8)
+    M, K = x.shape
+    N = Q.shape[0]
+    assert Q.shape == (N, K)
+    if B is None or A is None:
+        r = 0
+        B = A = None
+    else:
+        B = np.ascontiguousarray(B, dtype=np.uint16)
+        A = np.ascontiguousarray(A, dtype=np.uint16)
+        r = B.shape[0]
+        assert B.shape == (r, K) and A.shape == (N, r)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.uint16)
+        assert bias.shape == (N,)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int32)
+        nrows = rows.shape[0]
+    else:
+        nrows = M
+    y = np.empty((nrows, N), dtype=np.float64)
+    rc = lib().llo_forward(M, K, N, r, _ptr(x), _ptr(B), _ptr(A), _ptr(Q), _ptr(scale),
+                           int(scale_mode), _ptr(bias), int(mode), _ptr(rows), nrows,
+                           _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return y
+
+
+def forward_inputs(inp, mode=EXACT, rows=None):
+    """forward() on a synth_inputs.LayerInputs."""
+    from synth_inputs import to_numpy_bits
+    return forward(to_numpy_bits(inp.x), to_numpy_bits(inp.B), to_numpy_bits(inp.A),
+                   to_numpy_bits(inp.Q), to_numpy_bits(inp.scale), inp.scale_mode,
+                   to_numpy_bits(inp.bias), mode=mode, rows=rows)
+
+
+def tolerance_bound(y_ref: np.ndarray, rms: float | None = None) -> np.ndarray:
+    """Per-element acceptance bound |err| <= 8e-3*|y_ref| + 2e-3*RMS(y_ref),
+    RMS over the whole output tensor of the call (or the given value)."""
+    if rms is None:
+        rms = float(np.sqrt(np.mean(np.square(y_ref)))) if y_ref.size else 0.0
+    return 8e-3 * np.abs(y_ref) + 2e-3 * rms
