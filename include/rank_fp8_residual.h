@@ -1,0 +1,138 @@
+/*
+ * rank_fp8_residual.h -- C ABI of the B200 (sm_100a) LiteLinear forward.
+ *
+ * The layer stores a weight as a low-rank pair plus an FP8 residual and
+ * evaluates (LiteLinear README, introduction, the display formula):
+ *
+ *     W ~= A*B + Q_fp8,
+ *     y  = (x B^T) A^T + scale * (x Q_fp8^T) + bias
+ *
+ * Storage formats (README "Features"): A and B bf16, Q_fp8 e4m3fn (the
+ * NVIDIA variant), bf16 activations in and out (README "Usage").  Factor
+ * shapes as in SVDLinearLayer (tt_compressor page, class SVDLinearLayer:
+ * A is (out, r), B is (r, in)); Q is shaped like nn.Linear.weight.
+ *
+ *   x     [M, K]  bf16, row-major (K contiguous)
+ *   B     [r, K]  bf16, row-major
+ *   A     [N, r]  bf16, row-major
+ *   Q     [N, K]  e4m3fn codes, one byte each, row-major
+ *   scale [N] fp32 (LL_SCALE_PER_ROW, one per output feature) or [1] fp32
+ *         (LL_SCALE_PER_TENSOR).  It multiplies the x*Q^T term only (the
+ *         README's "scale"; its state-dict key is Q_scale_inv, and it is
+ *         applied as a multiplier).
+ *   bias  [N] bf16, or NULL for no bias
+ *   y     [M, N]  bf16, row-major
+ *
+ * All pointers passed to the compute calls are device pointers on the
+ * device that was current when the layer was created.  Every call is
+ * thread-compatible: one handle must not be used from two host threads at
+ * the same time, and a handle's forward calls must be ordered on one
+ * stream (they share the handle's workspace).  Distinct handles are
+ * independent.
+ *
+ * Error behaviour: every int-returning call returns LL_OK (0) or one of
+ * the LL_ERR_* codes below; ll_create returns NULL on error and records
+ * the code for ll_last_error().  Argument errors are reported
+ * synchronously and leave the handle unchanged.  Asynchronous device
+ * faults surface at the next synchronising CUDA call; a device-side wait
+ * that exceeded its time limit is reported by ll_status() after the
+ * stream has been synchronised.
+ */
+#ifndef RANK_FP8_RESIDUAL_H
+#define RANK_FP8_RESIDUAL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ll_layer *ll_handle;
+
+enum { LL_SCALE_PER_TENSOR = 0, LL_SCALE_PER_ROW = 1 };
+
+enum {
+  LL_OK = 0,
+  LL_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad size or mode */
+  LL_ERR_UNSUPPORTED = 2,    /* valid request this build does not handle */
+  LL_ERR_NOT_READY = 3,      /* forward before ll_set_weights succeeded */
+  LL_ERR_NAN_CODE = 4,       /* Q holds an e4m3fn NaN code (0x7F or 0xFF) */
+  LL_ERR_OOM = 5,            /* device allocation failed */
+  LL_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
+  LL_ERR_DEVICE_TIMEOUT = 7  /* a device-side wait ran past its limit */
+};
+
+/* Kernel variants for ll_set_variant. */
+enum { LL_VARIANT_AUTO = 0, LL_VARIANT_TC = 1 };
+
+/* Create a layer with N output features, K input features and rank r on
+ * the current CUDA device.  Requires N >= 1 and N % 8 == 0, K >= 16 and
+ * K % 16 == 0, 0 <= r <= 512, scale_mode one of LL_SCALE_*.  The handle is
+ * host-allocated; device memory for the factors is allocated here.
+ * Returns NULL on error (see ll_last_error()). */
+ll_handle ll_create(int N, int K, int r, int scale_mode);
+
+/* Copy the factors into handle-owned device memory (device-to-device;
+ * the caller may free its buffers once the call returns -- the call
+ * synchronises the device).  A: bf16 [N, r]; B: bf16 [r, K] (both may be
+ * NULL when r == 0); Q: e4m3fn codes [N, K]; scale: fp32 [N] or [1] by
+ * the layer's scale_mode; bias: bf16 [N] or NULL.  All non-NULL pointers
+ * must be 16-byte aligned device pointers except scale and bias (4- and
+ * 2-byte aligned).  The rank is zero-padded internally to a multiple of
+ * 64 (exact).  Returns LL_ERR_NAN_CODE if any Q code is 0x7F or 0xFF;
+ * LL_ERR_INVALID_ARG for null/misaligned/non-device pointers or a
+ * non-finite scale. */
+int ll_set_weights(ll_handle h, const void *A, const void *B, const void *Q, const float *scale,
+                   const void *bias);
+
+/* y = forward(x) for M rows on `stream` (a cudaStream_t; NULL is the
+ * legacy default stream).  x: bf16 [M, K], y: bf16 [M, N], both 16-byte
+ * aligned device pointers that must not overlap.  M == 0 is a no-op.  The
+ * call is asynchronous; x and y are borrowed until the stream reaches the
+ * end of the call.  The first call with a larger M than any before grows
+ * the handle's workspace with stream-ordered allocation (call ll_reserve
+ * beforehand to avoid that, e.g. before graph capture). */
+int ll_forward(ll_handle h, const void *x, void *y, int M, void *stream);
+
+/* ll_forward on HOST buffers: copies x (host, bf16 [M, K]) to the device,
+ * runs the forward and copies y back to the host (bf16 [M, N]), all on
+ * `stream`.  Pinned host buffers make the copies asynchronous; the caller
+ * synchronises the stream before reading y.  Device staging buffers are
+ * handle-owned and grown on demand. */
+int ll_forward_host(ll_handle h, const void *x_host, void *y_host, int M, void *stream);
+
+/* Pre-size the workspace for forwards of up to max_M rows (synchronous). */
+int ll_reserve(ll_handle h, int max_M);
+
+/* Select a kernel variant (LL_VARIANT_AUTO picks by M). */
+int ll_set_variant(ll_handle h, int variant);
+
+/* Device status word of the handle: LL_OK, or LL_ERR_DEVICE_TIMEOUT if a
+ * kernel of this handle gave up on a wait.  Synchronises the device;
+ * call after the stream of the forward has been synchronised.  Reading
+ * the status clears it. */
+int ll_status(ll_handle h);
+
+/* Debug controls: timeout_ns bounds every device-side wait (default 2 s);
+ * withhold_producer != 0 makes the main kernel's loader issue nothing, so
+ * its consumers run into the timeout (used to test the timeout path). */
+int ll_set_debug(ll_handle h, int withhold_producer, uint64_t timeout_ns);
+
+/* Release the handle and all device memory it owns (synchronises). */
+void ll_destroy(ll_handle h);
+
+/* Code of the last failed call on this host thread (LL_OK if none). */
+int ll_last_error(void);
+
+/* Static description of a status code. */
+const char *ll_status_string(int code);
+
+/* Number of kernels the last ll_forward on this handle launched. */
+int ll_last_launch_count(ll_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RANK_FP8_RESIDUAL_H */

@@ -1,0 +1,183 @@
+"""Python binding of the B200 LiteLinear forward library.
+
+Thin ctypes marshalling over the C ABI in include/rank_fp8_residual.h; every
+step of the forward runs in the library's CUDA kernels.  Functions keep the
+C names and accept either raw integers (device addresses, stream handles)
+or torch tensors / streams, from which they take ``data_ptr()`` and
+``cuda_stream``.  There is no CPU fallback: importing raises if the shared
+library has not been built (``python -m rank_fp8_residual_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librank_fp8_residual_b200.so")
+
+LL_SCALE_PER_TENSOR = 0
+LL_SCALE_PER_ROW = 1
+
+LL_OK = 0
+LL_ERR_INVALID_ARG = 1
+LL_ERR_UNSUPPORTED = 2
+LL_ERR_NOT_READY = 3
+LL_ERR_NAN_CODE = 4
+LL_ERR_OOM = 5
+LL_ERR_CUDA = 6
+LL_ERR_DEVICE_TIMEOUT = 7
+
+LL_VARIANT_AUTO = 0
+LL_VARIANT_TC = 1
+
+# Every symbol the header declares, with (restype, argtypes).
+_P = ctypes.c_void_p
+_SIGNATURES = {
+    "ll_create": (_P, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "ll_set_weights": (ctypes.c_int, [_P, _P, _P, _P, _P, _P]),
+    "ll_forward": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, _P]),
+    "ll_forward_host": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, _P]),
+    "ll_reserve": (ctypes.c_int, [_P, ctypes.c_int]),
+    "ll_set_variant": (ctypes.c_int, [_P, ctypes.c_int]),
+    "ll_status": (ctypes.c_int, [_P]),
+    "ll_set_debug": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_uint64]),
+    "ll_destroy": (None, [_P]),
+    "ll_last_error": (ctypes.c_int, []),
+    "ll_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ll_last_launch_count": (ctypes.c_int, [_P]),
+}
+
+
+class LLError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} (code {code})" if what else status_string(code))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m rank_fp8_residual_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _addr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def status_string(code: int) -> str:
+    return _lib.ll_status_string(int(code)).decode()
+
+
+def ll_last_error() -> int:
+    return _lib.ll_last_error()
+
+
+def ll_create(N: int, K: int, r: int, scale_mode: int) -> int:
+    h = _lib.ll_create(int(N), int(K), int(r), int(scale_mode))
+    if not h:
+        raise LLError(_lib.ll_last_error(), "ll_create")
+    return h
+
+
+def ll_set_weights(h: int, A, B, Q, scale, bias=None) -> None:
+    rc = _lib.ll_set_weights(h, _addr(A), _addr(B), _addr(Q), _addr(scale), _addr(bias))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_set_weights")
+
+
+def ll_forward(h: int, x, y, M: int, stream=None) -> None:
+    rc = _lib.ll_forward(h, _addr(x), _addr(y), int(M), _stream(stream))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_forward")
+
+
+def ll_forward_host(h: int, x_host, y_host, M: int, stream=None) -> None:
+    rc = _lib.ll_forward_host(h, _addr(x_host), _addr(y_host), int(M), _stream(stream))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_forward_host")
+
+
+def ll_reserve(h: int, max_M: int) -> None:
+    rc = _lib.ll_reserve(h, int(max_M))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_reserve")
+
+
+def ll_set_variant(h: int, variant: int) -> None:
+    rc = _lib.ll_set_variant(h, int(variant))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_set_variant")
+
+
+def ll_status(h: int) -> int:
+    return _lib.ll_status(h)
+
+
+def ll_set_debug(h: int, withhold_producer: bool, timeout_ns: int) -> None:
+    rc = _lib.ll_set_debug(h, int(bool(withhold_producer)), int(timeout_ns))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_set_debug")
+
+
+def ll_destroy(h: int) -> None:
+    _lib.ll_destroy(h)
+
+
+def ll_last_launch_count(h: int) -> int:
+    return _lib.ll_last_launch_count(h)
+
+
+class LiteLinearLayer:
+    """Owns one library handle; ``forward(x)`` returns a new bf16 tensor.
+
+    Tensors must be CUDA tensors on the current device: A bf16 [N,r],
+    B bf16 [r,K], Q uint8 (e4m3fn codes) [N,K], scale float32 [N] or [1],
+    bias bf16 [N] or None.
+    """
+
+    def __init__(self, N: int, K: int, r: int, scale_mode: int = LL_SCALE_PER_ROW):
+        self.N, self.K, self.r, self.scale_mode = N, K, r, scale_mode
+        self.handle = ll_create(N, K, r, scale_mode)
+
+    def set_weights(self, A, B, Q, scale, bias=None):
+        ll_set_weights(self.handle, A, B, Q, scale, bias)
+
+    def forward(self, x, out=None, stream=None):
+        import torch
+        M = x.shape[0]
+        if out is None:
+            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+        ll_forward(self.handle, x, out, M, stream)
+        return out
+
+    def close(self):
+        if self.handle:
+            ll_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,586 @@
+// Host side of the C ABI declared in include/rank_fp8_residual.h:
+// argument validation, handle-owned device copies of the factors, TMA
+// tensor-map construction, workspace management and the kernel chain of
+// one forward (see ll_kernels.cuh).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/rank_fp8_residual.h"
+#include "ll_kernels.cuh"
+
+namespace {
+
+thread_local int g_last_error = LL_OK;
+
+int fail(int code) {
+  g_last_error = code;
+  return code;
+}
+
+// ------------------------------------------------ driver entry point (TMA)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes per element, row pitch
+// `pitch_bytes`; box = {box_cols, box_rows}.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, uint64_t rows, uint64_t cols,
+              uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  (void)elem;
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+struct ll_layer {
+  int N = 0, K = 0, r = 0, r_pad = 0, scale_mode = 0;
+  int device = 0, num_sms = 0;
+  bool ready = false;
+  bool has_bias = false;
+  uint8_t* Q = nullptr;
+  uint16_t* A = nullptr;  // [N, r_pad]
+  uint16_t* B = nullptr;  // [r_pad, K]
+  float* scale = nullptr; // [N]
+  uint16_t* bias = nullptr;
+  int* status = nullptr;  // device status word
+  int* nanflag = nullptr;
+  // workspace for t
+  int ws_M = 0;
+  uint16_t* t_hi = nullptr;
+  uint16_t* t_lo = nullptr;
+  float* part = nullptr;
+  size_t part_bytes = 0;
+  // host-buffer forward staging
+  void* dx = nullptr;
+  void* dy = nullptr;
+  size_t dx_bytes = 0, dy_bytes = 0;
+  // weight tensor maps
+  CUtensorMap tm_q, tm_a, tm_b;
+  int rc = 64;
+  // per-call cache
+  const void* c_x = nullptr;
+  void* c_y = nullptr;
+  int c_M = -1;
+  CUtensorMap c_tm_x, c_tm_y, c_tm_thi, c_tm_tlo;
+  int variant = LL_VARIANT_AUTO;
+  int withhold = 0;
+  uint64_t timeout_ns = 2000000000ull;
+  int last_launches = 0;
+};
+
+namespace {
+
+void free_layer_mem(ll_layer* h) {
+  cudaFree(h->Q);
+  cudaFree(h->A);
+  cudaFree(h->B);
+  cudaFree(h->scale);
+  cudaFree(h->bias);
+  cudaFree(h->status);
+  cudaFree(h->nanflag);
+  cudaFree(h->t_hi);
+  cudaFree(h->t_lo);
+  cudaFree(h->part);
+  cudaFree(h->dx);
+  cudaFree(h->dy);
+}
+
+int set_smem_attrs_once() {
+  static int rc = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    rc = 0;
+    if (cudaFuncSetAttribute(llk::ll_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::main_smem_bytes()) != cudaSuccess)
+      rc = 1;
+    if (cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::lr_smem_bytes(256)) != cudaSuccess)
+      rc = 1;
+  });
+  return rc;
+}
+
+// Grow the t workspace to hold `M` rows (stream-ordered).
+int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
+  if (h->r_pad == 0) return LL_OK;
+  if (M > h->ws_M) {
+    int newM = std::max(M, h->ws_M * 3 / 2);
+    newM = (newM + 127) / 128 * 128;
+    uint16_t *th = nullptr, *tl = nullptr;
+    const size_t bytes = static_cast<size_t>(newM) * h->r_pad * sizeof(uint16_t);
+    if (cudaMallocAsync(reinterpret_cast<void**>(&th), bytes, st) != cudaSuccess ||
+        cudaMallocAsync(reinterpret_cast<void**>(&tl), bytes, st) != cudaSuccess) {
+      cudaGetLastError();
+      if (th) cudaFreeAsync(th, st);
+      return LL_ERR_OOM;
+    }
+    if (h->t_hi) cudaFreeAsync(h->t_hi, st);
+    if (h->t_lo) cudaFreeAsync(h->t_lo, st);
+    h->t_hi = th;
+    h->t_lo = tl;
+    h->ws_M = newM;
+    h->c_M = -1;  // invalidate maps over t
+  }
+  if (part_need > h->part_bytes) {
+    float* pp = nullptr;
+    const size_t nb = std::max(part_need, h->part_bytes * 3 / 2);
+    if (cudaMallocAsync(reinterpret_cast<void**>(&pp), nb, st) != cudaSuccess) {
+      cudaGetLastError();
+      return LL_ERR_OOM;
+    }
+    if (h->part) cudaFreeAsync(h->part, st);
+    h->part = pp;
+    h->part_bytes = nb;
+  }
+  return LL_OK;
+}
+
+struct LrPlan {
+  int rc, ksplit, kb_per_split, m_tiles, r_chunks;
+};
+
+LrPlan plan_lowrank(const ll_layer* h, int M) {
+  LrPlan p{};
+  const int nK = (h->K + llk::kBK - 1) / llk::kBK;
+  p.m_tiles = (M + 127) / 128;
+  if (h->r_pad == 0) {  // no low-rank term: nothing to plan
+    p.rc = 64;
+    p.ksplit = 1;
+    p.kb_per_split = nK;
+    p.r_chunks = 0;
+    return p;
+  }
+  // Column block of t per CTA: the widest of 256/128/64 that divides r_pad
+  // (TMEM allocations are powers of two); 128 when the token count alone
+  // cannot occupy half the GPU, so that more CTAs share the read of B.
+  p.rc = (h->r_pad % 256 == 0) ? 256 : (h->r_pad % 128 == 0) ? 128 : 64;
+  if (p.rc == 256 && p.m_tiles * (h->r_pad / 128) <= h->num_sms / 2) p.rc = 128;
+  p.r_chunks = h->r_pad / p.rc;
+  const int ctas = p.m_tiles * p.r_chunks;
+  int ks = std::max(1, h->num_sms / ctas);
+  ks = std::min(ks, nK);
+  p.kb_per_split = (nK + ks - 1) / ks;
+  p.ksplit = (nK + p.kb_per_split - 1) / p.kb_per_split;
+  return p;
+}
+
+size_t part_bytes_for(const ll_layer* h, int M) {
+  const LrPlan p = plan_lowrank(h, M);
+  return p.ksplit > 1 ? static_cast<size_t>(p.ksplit) * M * h->r_pad * sizeof(float) : 0;
+}
+
+bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
+  if (h->c_x == x && h->c_y == y && h->c_M == M) return true;
+  using namespace llk;
+  if (!make_map(&h->c_tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->K, 2ull * h->K, kBK, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
+  if (!make_map(&h->c_tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->N, 2ull * h->N, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  if (h->r_pad > 0) {
+    if (!make_map(&h->c_tm_thi, h->t_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->r_pad, 2ull * h->r_pad, kBK,
+                  128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+    if (!make_map(&h->c_tm_tlo, h->t_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->r_pad, 2ull * h->r_pad, kBK,
+                  128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  h->c_x = x;
+  h->c_y = y;
+  h->c_M = M;
+  return true;
+}
+
+int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) {
+  using namespace llk;
+  h->last_launches = 0;
+  const LrPlan lp = plan_lowrank(h, M);
+  int rc = ensure_workspace(h, M, st, lp.ksplit > 1 ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0);
+  if (rc != LL_OK) return rc;
+  if (!build_call_maps(h, x, y, M)) return LL_ERR_CUDA;
+  const Watch watch{h->status, h->timeout_ns};
+  int launches = 0;
+
+  if (h->r_pad > 0) {
+    LrDownParams lpp;
+    lpp.tm_x = h->c_tm_x;
+    // B map for the chosen column block height.
+    if (lp.rc != h->rc) {
+      if (!make_map(&h->tm_b, h->B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->r_pad, h->K, 2ull * h->K, kBK, lp.rc,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+        return LL_ERR_CUDA;
+      h->rc = lp.rc;
+    }
+    lpp.tm_b = h->tm_b;
+    lpp.t_hi = h->t_hi;
+    lpp.t_lo = h->t_lo;
+    lpp.part = h->part;
+    lpp.M = M;
+    lpp.K = h->K;
+    lpp.r_pad = h->r_pad;
+    lpp.rc = lp.rc;
+    lpp.ksplit = lp.ksplit;
+    lpp.kb_per_split = lp.kb_per_split;
+    lpp.watch = watch;
+    dim3 grid(lp.m_tiles, lp.r_chunks, lp.ksplit);
+    ll_lrdown_kernel<<<grid, kLrThreads, lr_smem_bytes(lp.rc), st>>>(lpp);
+    ++launches;
+    if (lp.ksplit > 1) {
+      const size_t total4 = static_cast<size_t>(M) * h->r_pad / 4;
+      int blocks = static_cast<int>(std::min<size_t>((total4 + 255) / 256, static_cast<size_t>(h->num_sms) * 4));
+      ll_lrsplit_kernel<<<blocks, 256, 0, st>>>(h->part, h->t_hi, h->t_lo, M, h->r_pad, lp.ksplit);
+      ++launches;
+    }
+    if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
+  }
+
+  MainParams mp;
+  mp.tm_x = h->c_tm_x;
+  mp.tm_q = h->tm_q;
+  mp.tm_a = h->tm_a;
+  mp.tm_thi = h->c_tm_thi;
+  mp.tm_tlo = h->c_tm_tlo;
+  mp.tm_y = h->c_tm_y;
+  mp.scale = h->scale;
+  mp.bias = h->has_bias ? h->bias : nullptr;
+  mp.M = M;
+  mp.N = h->N;
+  mp.K = h->K;
+  mp.r_pad = h->r_pad;
+  mp.n_ftiles = (h->N + 127) / 128;
+  mp.n_ttiles = (M + 127) / 128;
+  mp.lr_from_primary = h->r_pad > 0 ? 1 : 0;
+  mp.withhold = h->withhold;
+  mp.watch = watch;
+  const int tiles = mp.n_ftiles * mp.n_ttiles;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(tiles, h->num_sms));
+  cfg.blockDim = dim3(kMainThreads);
+  cfg.dynamicSmemBytes = main_smem_bytes();
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = h->r_pad > 0 ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, ll_main_kernel, mp) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
+  ++launches;
+  h->last_launches = launches;
+  return LL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ll_status_string(int code) {
+  switch (code) {
+    case LL_OK: return "ok";
+    case LL_ERR_INVALID_ARG: return "invalid argument";
+    case LL_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LL_ERR_NOT_READY: return "weights not set";
+    case LL_ERR_NAN_CODE: return "residual holds an e4m3fn NaN code";
+    case LL_ERR_OOM: return "device allocation failed";
+    case LL_ERR_CUDA: return "CUDA call failed";
+    case LL_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int ll_last_error(void) { return g_last_error; }
+
+ll_handle ll_create(int N, int K, int r, int scale_mode) {
+  g_last_error = LL_OK;
+  if (N < 1 || K < 16 || r < 0 || (N % 8) != 0 || (K % 16) != 0 ||
+      (scale_mode != LL_SCALE_PER_TENSOR && scale_mode != LL_SCALE_PER_ROW)) {
+    fail(LL_ERR_INVALID_ARG);
+    return nullptr;
+  }
+  if (r > 512) {
+    fail(LL_ERR_UNSUPPORTED);
+    return nullptr;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    fail(LL_ERR_CUDA);
+    return nullptr;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+    cudaGetLastError();
+    fail(LL_ERR_CUDA);
+    return nullptr;
+  }
+  if (prop.major != 10 || prop.minor != 0) {  // built for sm_100a only
+    fail(LL_ERR_UNSUPPORTED);
+    return nullptr;
+  }
+  if (set_smem_attrs_once() != 0 || !encode_fn()) {
+    fail(LL_ERR_CUDA);
+    return nullptr;
+  }
+  ll_layer* h = new ll_layer();
+  h->N = N;
+  h->K = K;
+  h->r = r;
+  h->r_pad = (r + 63) / 64 * 64;
+  h->scale_mode = scale_mode;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  bool ok = true;
+  ok &= cudaMalloc(&h->Q, static_cast<size_t>(N) * K) == cudaSuccess;
+  ok &= cudaMalloc(&h->scale, sizeof(float) * N) == cudaSuccess;
+  ok &= cudaMalloc(&h->bias, sizeof(uint16_t) * N) == cudaSuccess;
+  ok &= cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
+  ok &= cudaMalloc(&h->nanflag, sizeof(int)) == cudaSuccess;
+  if (h->r_pad > 0) {
+    ok &= cudaMalloc(&h->A, sizeof(uint16_t) * N * static_cast<size_t>(h->r_pad)) == cudaSuccess;
+    ok &= cudaMalloc(&h->B, sizeof(uint16_t) * static_cast<size_t>(h->r_pad) * K) == cudaSuccess;
+  }
+  if (!ok) {
+    cudaGetLastError();
+    free_layer_mem(h);
+    delete h;
+    fail(LL_ERR_OOM);
+    return nullptr;
+  }
+  cudaMemset(h->status, 0, sizeof(int));
+  using namespace llk;
+  ok &= make_map(&h->tm_q, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (h->r_pad > 0) {
+    ok &= make_map(&h->tm_a, h->A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, h->r_pad, 2ull * h->r_pad, kBK, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    h->rc = std::min(h->r_pad, 256);
+    ok &= make_map(&h->tm_b, h->B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->r_pad, K, 2ull * K, kBK, h->rc,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (!ok) {
+    free_layer_mem(h);
+    delete h;
+    fail(LL_ERR_CUDA);
+    return nullptr;
+  }
+  return h;
+}
+
+int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, const float* scale,
+                   const void* bias) {
+  g_last_error = LL_OK;
+  if (!h || !Q || !scale) return fail(LL_ERR_INVALID_ARG);
+  if (h->r > 0 && (!A || !B)) return fail(LL_ERR_INVALID_ARG);
+  if (!is_device_ptr(Q) || !is_device_ptr(scale) || (bias && !is_device_ptr(bias)) ||
+      (h->r > 0 && (!is_device_ptr(A) || !is_device_ptr(B))))
+    return fail(LL_ERR_INVALID_ARG);
+  if (!aligned(Q, 16) || !aligned(scale, 4) || (bias && !aligned(bias, 2)) ||
+      (h->r > 0 && (!aligned(A, 2) || !aligned(B, 2))))
+    return fail(LL_ERR_INVALID_ARG);
+  const int N = h->N, K = h->K, r = h->r, rp = h->r_pad;
+  // scale must be finite
+  const int ns = h->scale_mode == LL_SCALE_PER_ROW ? N : 1;
+  std::vector<float> hs(ns);
+  if (cudaMemcpy(hs.data(), scale, sizeof(float) * ns, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  for (float v : hs)
+    if (!std::isfinite(v)) return fail(LL_ERR_INVALID_ARG);
+  // NaN-code scan of the residual (before touching the handle's copy).
+  if (cudaMemset(h->nanflag, 0, sizeof(int)) != cudaSuccess) return fail(LL_ERR_CUDA);
+  const size_t nq = static_cast<size_t>(N) * K;
+  llk::ll_nan_scan_kernel<<<std::max(1, std::min(h->num_sms * 8, static_cast<int>((nq / 16 + 255) / 256))), 256>>>(
+      static_cast<const uint8_t*>(Q), nq, h->nanflag);
+  int flag = 0;
+  if (cudaGetLastError() != cudaSuccess ||
+      cudaMemcpy(&flag, h->nanflag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  if (flag) return fail(LL_ERR_NAN_CODE);
+  bool ok = true;
+  ok &= cudaMemcpy(h->Q, Q, nq, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  if (h->scale_mode == LL_SCALE_PER_ROW) {
+    ok &= cudaMemcpy(h->scale, scale, sizeof(float) * N, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  } else {
+    std::vector<float> full(N, hs[0]);
+    ok &= cudaMemcpy(h->scale, full.data(), sizeof(float) * N, cudaMemcpyHostToDevice) == cudaSuccess;
+  }
+  if (bias) {
+    ok &= cudaMemcpy(h->bias, bias, sizeof(uint16_t) * N, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  } else {
+    ok &= cudaMemset(h->bias, 0, sizeof(uint16_t) * N) == cudaSuccess;
+  }
+  h->has_bias = bias != nullptr;
+  if (rp > 0) {
+    ok &= cudaMemset(h->A, 0, sizeof(uint16_t) * N * static_cast<size_t>(rp)) == cudaSuccess;
+    ok &= cudaMemset(h->B, 0, sizeof(uint16_t) * static_cast<size_t>(rp) * K) == cudaSuccess;
+    ok &= cudaMemcpy2D(h->A, sizeof(uint16_t) * rp, A, sizeof(uint16_t) * r, sizeof(uint16_t) * r, N,
+                       cudaMemcpyDeviceToDevice) == cudaSuccess;
+    ok &= cudaMemcpy(h->B, B, sizeof(uint16_t) * static_cast<size_t>(r) * K, cudaMemcpyDeviceToDevice) ==
+          cudaSuccess;
+  }
+  ok &= cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    h->ready = false;
+    return fail(LL_ERR_CUDA);
+  }
+  h->ready = true;
+  return LL_OK;
+}
+
+int ll_forward(ll_handle h, const void* x, void* y, int M, void* stream) {
+  g_last_error = LL_OK;
+  if (!h) return fail(LL_ERR_INVALID_ARG);
+  if (M < 0) return fail(LL_ERR_INVALID_ARG);
+  if (!h->ready) return fail(LL_ERR_NOT_READY);
+  if (M == 0) {
+    h->last_launches = 0;
+    return LL_OK;
+  }
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return fail(LL_ERR_INVALID_ARG);
+  const char* xb = static_cast<const char*>(x);
+  const char* yb = static_cast<const char*>(y);
+  const size_t xs = static_cast<size_t>(M) * h->K * 2, ys = static_cast<size_t>(M) * h->N * 2;
+  if (xb < yb + ys && yb < xb + xs) return fail(LL_ERR_INVALID_ARG);
+  int rc = forward_device(h, x, y, M, static_cast<cudaStream_t>(stream));
+  return rc == LL_OK ? LL_OK : fail(rc);
+}
+
+int ll_forward_host(ll_handle h, const void* x_host, void* y_host, int M, void* stream) {
+  g_last_error = LL_OK;
+  if (!h) return fail(LL_ERR_INVALID_ARG);
+  if (M < 0 || (M > 0 && (!x_host || !y_host))) return fail(LL_ERR_INVALID_ARG);
+  if (!h->ready) return fail(LL_ERR_NOT_READY);
+  if (M == 0) return LL_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t xs = static_cast<size_t>(M) * h->K * 2, ys = static_cast<size_t>(M) * h->N * 2;
+  if (xs > h->dx_bytes) {
+    void* p = nullptr;
+    if (cudaMallocAsync(&p, xs, st) != cudaSuccess) { cudaGetLastError(); return fail(LL_ERR_OOM); }
+    if (h->dx) cudaFreeAsync(h->dx, st);
+    h->dx = p;
+    h->dx_bytes = xs;
+  }
+  if (ys > h->dy_bytes) {
+    void* p = nullptr;
+    if (cudaMallocAsync(&p, ys, st) != cudaSuccess) { cudaGetLastError(); return fail(LL_ERR_OOM); }
+    if (h->dy) cudaFreeAsync(h->dy, st);
+    h->dy = p;
+    h->dy_bytes = ys;
+  }
+  if (cudaMemcpyAsync(h->dx, x_host, xs, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  int rc = forward_device(h, h->dx, h->dy, M, st);
+  if (rc != LL_OK) return fail(rc);
+  if (cudaMemcpyAsync(y_host, h->dy, ys, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  return LL_OK;
+}
+
+int ll_reserve(ll_handle h, int max_M) {
+  g_last_error = LL_OK;
+  if (!h || max_M < 0) return fail(LL_ERR_INVALID_ARG);
+  // The partial-sum buffer is largest at the biggest M of each tile count.
+  size_t need = 0;
+  for (int m = 128; m - 128 < max_M; m += 128) need = std::max(need, part_bytes_for(h, std::min(m, max_M)));
+  int rc = ensure_workspace(h, max_M, 0, need);
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    rc = LL_ERR_CUDA;
+  }
+  return rc == LL_OK ? LL_OK : fail(rc);
+}
+
+int ll_set_variant(ll_handle h, int variant) {
+  g_last_error = LL_OK;
+  if (!h || (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC)) return fail(LL_ERR_INVALID_ARG);
+  h->variant = variant;
+  return LL_OK;
+}
+
+int ll_status(ll_handle h) {
+  g_last_error = LL_OK;
+  if (!h) return fail(LL_ERR_INVALID_ARG);
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  if (v != 0) {
+    cudaMemset(h->status, 0, sizeof(int));
+    cudaDeviceSynchronize();
+    return LL_ERR_DEVICE_TIMEOUT;
+  }
+  return LL_OK;
+}
+
+int ll_set_debug(ll_handle h, int withhold_producer, uint64_t timeout_ns) {
+  g_last_error = LL_OK;
+  if (!h || timeout_ns == 0) return fail(LL_ERR_INVALID_ARG);
+  h->withhold = withhold_producer ? 1 : 0;
+  h->timeout_ns = timeout_ns;
+  return LL_OK;
+}
+
+int ll_last_launch_count(ll_handle h) { return h ? h->last_launches : 0; }
+
+void ll_destroy(ll_handle h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  free_layer_mem(h);
+  cudaGetLastError();
+  delete h;
+}
+
+}  // extern "C"

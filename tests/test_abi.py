@@ -1,0 +1,87 @@
+"""The C-ABI library loads and exports every function include/*.h declares;
+host-side argument checks reject bad calls before touching a GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"\b(ll_[a-z_0-9]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("ll_create", "ll_set_weights", "ll_forward", "ll_destroy", "ll_last_error",
+              "ll_status_string", "ll_status", "ll_forward_host", "ll_reserve"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import rank_fp8_residual_b200 as ll
+    lib = ctypes.CDLL(ll.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding wraps every declared function under the same name
+    for n in _declared_functions():
+        assert n in ll._SIGNATURES, n
+
+
+def test_status_strings():
+    import rank_fp8_residual_b200 as ll
+    assert ll.status_string(ll.LL_OK) == "ok"
+    assert "NaN" in ll.status_string(ll.LL_ERR_NAN_CODE)
+    assert ll.status_string(12345) == "unknown status"
+
+
+@pytest.mark.parametrize("N,K,r,mode", [(7, 64, 4, 1), (8, 15, 4, 1), (8, 64, -1, 1),
+                                          (8, 64, 4, 2), (0, 64, 4, 1), (8, 0, 0, 0)])
+def test_create_rejects_bad_shapes_without_a_gpu(N, K, r, mode):
+    import rank_fp8_residual_b200 as ll
+    with pytest.raises(ll.LLError) as e:
+        ll.ll_create(N, K, r, mode)
+    assert e.value.code == ll.LL_ERR_INVALID_ARG
+
+
+def test_create_rank_above_limit_is_unsupported():
+    import rank_fp8_residual_b200 as ll
+    with pytest.raises(ll.LLError) as e:
+        ll.ll_create(64, 64, 513, 1)
+    assert e.value.code == ll.LL_ERR_UNSUPPORTED
+
+
+def test_null_handle_calls_fail_cleanly():
+    import rank_fp8_residual_b200 as ll
+    lib = ll._lib
+    assert lib.ll_forward(None, None, None, 4, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_last_error() == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_set_weights(None, None, None, None, None, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_forward_host(None, None, None, 1, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_reserve(None, 4) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_set_variant(None, 0) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_set_debug(None, 0, 1) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_last_launch_count(None) == 0
+    lib.ll_destroy(None)
+
+
+def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):
+    """Importing the binding without the built library raises."""
+    import importlib.util
+    import sys
+    src = os.path.join(ROOT, "rank_fp8_residual_b200", "__init__.py")
+    pkg = tmp_path / "rank_fp8_residual_b200"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(open(src).read())
+    spec = importlib.util.spec_from_file_location("llcopy", str(pkg / "__init__.py"))
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,182 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bar (per element): |y_gpu - y_ref| <= 8e-3*|y_ref| + 2e-3*RMS(y_ref), with
+y_ref the binary64 oracle of y = (x B^T) A^T + scale * (x Q^T) + bias
+(LiteLinear README, introduction) and RMS over the output of the call (over
+the sampled rows where only rows are sampled).  The widening check is exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rank_fp8_residual_b200 as ll
+from synth_inputs import (SCALE_PER_ROW, SCALE_PER_TENSOR, WORKLOADS, LayerInputs, make_inputs)
+
+from llgpu import DeviceLayer, check, run
+
+pytestmark = pytest.mark.gpu
+
+
+def _full(inp, what):
+    y = run(inp)
+    return check(y, oracle.forward_inputs(inp), what=what)
+
+
+def test_widening_is_exact_for_every_code():
+    """One-hot tokens pick single residual codes: y[m, n] = Q[n, m] exactly.
+    Every non-NaN code appears in every K position, so the swizzled shared
+    memory reads and the TMEM lane mapping are covered too."""
+    K = N = M = 256
+    n = torch.arange(N).view(N, 1)
+    k = torch.arange(K).view(1, K)
+    codes = ((n + k) % 256).to(torch.uint8)
+    codes[(codes == 0x7F) | (codes == 0xFF)] = 0
+    x = torch.eye(M, K, dtype=torch.bfloat16)
+    inp = LayerInputs(M, K, N, 0, SCALE_PER_TENSOR, x, None, None, codes,
+                      torch.ones(1, dtype=torch.float32), None)
+    y = run(inp).to(torch.float64)
+    expect = codes.view(torch.float8_e4m3fn).to(torch.float64).t()  # [M=K, N]
+    assert torch.equal(y, expect)
+
+
+def test_tiny_config():
+    _full(WORKLOADS["tiny_m64_k256_n256_r16"].inputs(), "tiny")
+
+
+@pytest.mark.parametrize("M,K,N,r", [(300, 272, 392, 40), (129, 1024, 136, 64), (517, 384, 1000, 200)])
+def test_ragged_multi_tile(M, K, N, r):
+    inp = make_inputs(M, K, N, r, scale_range=(1e-3, 3e-3), seed=M)
+    _full(inp, f"ragged {M}x{K}x{N} r{r}")
+
+
+def test_rank_zero():
+    _full(make_inputs(200, 256, 256, 0, seed=1), "r=0")
+
+
+def test_residual_zero_is_low_rank_only():
+    _full(make_inputs(200, 256, 256, 32, seed=2, q_zero=True), "Q=0")
+
+
+def test_per_tensor_scale_and_no_bias():
+    _full(make_inputs(150, 320, 264, 24, scale_mode=SCALE_PER_TENSOR, bias=False, seed=3),
+          "per-tensor, no bias")
+
+
+@pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 31, 64])
+def test_small_token_counts(M):
+    _full(make_inputs(M, 512, 1024, 96, seed=10 + M), f"M={M}")
+
+
+@pytest.mark.parametrize("M", [127, 128, 129, 255, 257])
+def test_token_tile_edges(M):
+    _full(make_inputs(M, 128, 256, 16, seed=20 + M), f"M={M}")
+
+
+@pytest.mark.parametrize("r", [1, 63, 64, 65, 128, 256, 320, 512])
+def test_rank_edges(r):
+    _full(make_inputs(140, 256, 256, r, seed=30 + r), f"r={r}")
+
+
+def test_attention_projection_full():
+    _full(WORKLOADS["attn_m3630_k2048_n2048_r32"].inputs(), "attn_m3630_k2048_n2048_r32")
+
+
+def _sampled_rows(M, n=48):
+    rng = np.random.default_rng(M)
+    rows = set(rng.choice(M, size=min(M, n), replace=False).tolist())
+    rows |= {0, M - 1, (M - 1) // 128 * 128}  # first, last, first row of the last tile
+    return sorted(rows)
+
+
+def _sampled(name):
+    inp = WORKLOADS[name].inputs()
+    y = run(inp)
+    rows = _sampled_rows(inp.M)
+    ref = oracle.forward_inputs(inp, rows=rows)
+    return check(y[rows], ref, what=name + " (sampled rows)")
+
+
+@pytest.mark.parametrize("name", ["ffn_up_m3630_k2048_n8192_r64", "ffn_down_m3630_k8192_n2048_r64"])
+def test_ffn_pair_sampled(name):
+    _sampled(name)
+
+
+@pytest.mark.parametrize("name", ["small_m1_k4096_n16384_r512", "small_m16_k4096_n16384_r512",
+                                  "small_m64_k4096_n16384_r512"])
+def test_small_batch_full(name):
+    _full(WORKLOADS[name].inputs(), name)
+
+
+@pytest.mark.parametrize("name", ["sweep_m1024_k4096_n4096_r32", "sweep_m4096_k4096_n16384_r512",
+                                  "sweep_m16384_k4096_n16384_r64"])
+def test_sweep_sampled(name):
+    _sampled(name)
+
+
+def test_repeated_calls_are_bitwise_identical():
+    inp = make_inputs(700, 512, 640, 64, seed=40)
+    d = DeviceLayer(inp)
+    try:
+        a = d.forward(inp.x)
+        b = d.forward(inp.x)
+        assert torch.equal(a, b)
+    finally:
+        d.close()
+
+
+def test_forward_host_matches_device():
+    inp = make_inputs(333, 256, 264, 32, seed=41)
+    d = DeviceLayer(inp)
+    try:
+        y_dev = d.forward(inp.x).cpu()
+        xh = inp.x.contiguous().pin_memory()
+        yh = torch.empty(inp.M, inp.N, dtype=torch.bfloat16).pin_memory()
+        ll.ll_forward_host(d.h, xh.data_ptr(), yh.data_ptr(), inp.M, None)
+        torch.cuda.synchronize()
+        assert torch.equal(yh, y_dev)
+    finally:
+        d.close()
+
+
+def test_set_weights_rejects_nan_codes():
+    inp = make_inputs(8, 64, 64, 8, seed=42)
+    inp.Q[3, 5] = 0xFF
+    h = ll.ll_create(64, 64, 8, SCALE_PER_ROW)
+    try:
+        with pytest.raises(ll.LLError) as e:
+            ll.ll_set_weights(h, inp.A.cuda(), inp.B.cuda(), inp.Q.cuda(), inp.scale.cuda(),
+                              inp.bias.cuda())
+        assert e.value.code == ll.LL_ERR_NAN_CODE
+        x = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(8, 64, dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(ll.LLError) as e:
+            ll.ll_forward(h, x, y, 8)
+        assert e.value.code == ll.LL_ERR_NOT_READY
+    finally:
+        ll.ll_destroy(h)
+
+
+def test_argument_errors_on_device():
+    inp = make_inputs(8, 64, 64, 8, seed=43)
+    d = DeviceLayer(inp)
+    try:
+        x = torch.zeros(9, 64, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(9, 64, dtype=torch.bfloat16, device="cuda")
+        for args, code in [((x, y, -1), ll.LL_ERR_INVALID_ARG),
+                           ((x.view(-1)[1:].data_ptr(), y, 4), ll.LL_ERR_INVALID_ARG),  # misaligned
+                           ((x, x, 4), ll.LL_ERR_INVALID_ARG)]:                          # overlap
+            with pytest.raises(ll.LLError) as e:
+                ll.ll_forward(d.h, *args)
+            assert e.value.code == code
+        ll.ll_forward(d.h, x, y, 0)  # M == 0 is a no-op
+        bad = inp.scale.clone()
+        bad[0] = float("inf")
+        with pytest.raises(ll.LLError) as e:
+            ll.ll_set_weights(d.h, d.A, d.B, d.Q, bad.cuda(), d.bias)
+        assert e.value.code == ll.LL_ERR_INVALID_ARG
+        with pytest.raises(ll.LLError) as e:  # host pointer where a device pointer is required
+            ll.ll_set_weights(d.h, d.A, d.B, inp.Q.data_ptr(), d.scale, d.bias)
+        assert e.value.code == ll.LL_ERR_INVALID_ARG
+    finally:
+        d.close()
