@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the LiteLinear forward ``ll_forward`` on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step = one ``ll_forward`` (every kernel of the path) over one batch of
+synthetic tokens for the named layer shape (default: the attention
+projection of a 480x704x81 video latent, M=3630 tokens, K=N=2048, r=32).
+Metric: algorithmic TFLOP/s, F = 2*M*(K*N + r*K + r*N) per step.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+device synchronise on both sides; each step is bracketed by CUDA events on
+the launching stream and L2 is flushed (a 256 MiB write) between steps,
+outside the events.  Multi-GPU (torchrun): each rank runs its own batch of
+M tokens against its own copy of the factors (token-sharded replicas, no
+data-path collective); the reported time is the max over ranks and the
+value counts the tokens of all ranks (weak scaling).
+
+Also reported on the same JSON line: ``e2e`` (same metric through
+``ll_forward_host`` with pinned host buffers, the H2D copy of x and the
+D2H copy of y inside each timed step), ``roofline`` for the dominant kernel
+(per-kernel device times from the library's profiling mode), ``clocks``
+(NVML samples taken during the timed region), ``gpu_launches`` and, on
+rank 0 at N=1, ``cpu_baseline`` (the fp64 CPU oracle on a row sample).
+
+``--impl reference`` times the CPU oracle instead (the reference arm of
+this build) on the same workload, metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synth_inputs import SCALE_PER_ROW, WORKLOADS  # noqa: E402
+
+DEFAULT_WORKLOAD = "attn_m3630_k2048_n2048_r32"
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def work_of(w, M=None):
+    M = w.M if M is None else M
+    K, N, r = w.K, w.N, w.r
+    flops = 2.0 * M * (K * N + r * K + r * N)
+    bytes_ = 2.0 * M * K + N * K + 2.0 * N * r + 2.0 * r * K + 4.0 * N + 2.0 * N + 2.0 * M * N
+    # the fused kernel (x Q^T and the up-projection; B is read by the
+    # down-projection kernel only)
+    main_flops = 2.0 * M * N * (K + r)
+    main_bytes = bytes_ - 2.0 * r * K
+    return flops, bytes_, main_flops, main_bytes
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rank_fp8_residual_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, or None when the
+    kernel sources changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, period_s=0.002):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return
+        self._t = threading.Thread(target=self._run, args=(period_s,), daemon=True)
+
+    def _run(self, period):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                self.reasons |= fn(self._h)
+            except Exception:
+                pass
+            time.sleep(period)
+
+    def start(self):
+        if self.ok:
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable" if not self.ok else "nvml"}
+        names = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples), "source": "nvml"}
+
+
+def cpu_baseline(w, budget_s=8.0):
+    """The fp64 oracle, as it stands, on a bounded row sample of the
+    workload, in the bench's unit (algorithmic TFLOP/s)."""
+    import oracle
+    inp = w.inputs()
+    probe = max(1, min(w.M, 16))
+    rows = list(range(probe))
+    t0 = time.perf_counter()
+    oracle.forward_inputs(inp, rows=rows)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(w.M, max(probe, probe * budget_s / dt)))
+    step = max(1, w.M // n)
+    rows = list(range(0, w.M, step))[:n]
+    t0 = time.perf_counter()
+    oracle.forward_inputs(inp, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = work_of(w, M=len(rows))[0]
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} of {w.M} token rows (every {step}th), full N={w.N}, "
+                      f"{dt:.2f} s wall"}
+
+
+def run_reference(args, w):
+    """Reference arm: the CPU oracle timed step by step on a row sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    inp = w.inputs()
+    probe = list(range(min(w.M, 8)))
+    t0 = time.perf_counter()
+    oracle.forward_inputs(inp, rows=probe)
+    per_row = max((time.perf_counter() - t0) / len(probe), 1e-7)
+    # each step ~0.5 s so that warm-up + steps stay within a few minutes
+    nrows = int(max(1, min(w.M, 0.5 / per_row)))
+    stride = max(1, w.M // nrows)
+    for i in range(args.warmup):
+        oracle.forward_inputs(inp, rows=list(range(i % stride, w.M, stride))[:nrows])
+    times = []
+    for i in range(args.steps):
+        rows = list(range(i % stride, w.M, stride))[:nrows]
+        t0 = time.perf_counter()
+        oracle.forward_inputs(inp, rows=rows)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    flops = work_of(w, M=nrows)[0]
+    value = args.steps * flops / total / 1e12
+    sample = f"{nrows} of {w.M} token rows per step (stride {stride}), full N={w.N}"
+    line = {
+        "impl": "reference", "metric": "ll_forward TFLOP/s (algorithmic)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "r": w.r,
+                   "scale_mode": "per_row" if w.scale_mode == SCALE_PER_ROW else "per_tensor"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import rank_fp8_residual_b200 as ll
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # Factors are shared (seed 0); each rank draws its own tokens.
+    inp = w.inputs(seed=0)
+    if rank != 0:
+        from synth_inputs import make_x
+        inp.x = make_x(w.M, w.K, seed=1000 + rank)
+    layer = ll.LiteLinearLayer(w.N, w.K, w.r, w.scale_mode)
+    layer.set_weights(inp.A.to(dev) if inp.A is not None else None,
+                      inp.B.to(dev) if inp.B is not None else None,
+                      inp.Q.to(dev), inp.scale.to(dev),
+                      inp.bias.to(dev) if inp.bias is not None else None)
+    h = layer.handle
+    ll.ll_reserve(h, w.M)
+    x = inp.x.to(dev)
+    y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    flops, bytes_, main_flops, main_bytes = work_of(w)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # --------------------------------------------------- device-timed steps
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            ll.ll_forward(h, x, y, w.M, stream)
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        launches = 0
+        sampler = ClockSampler(local_rank)
+        barrier()
+        torch.cuda.synchronize()
+        sampler.start()
+        for i in range(args.steps):
+            flush.zero_()
+            ev0[i].record(stream)
+            ll.ll_forward(h, x, y, w.M, stream)
+            ev1[i].record(stream)
+            launches += ll.ll_last_launch_count(h)
+        torch.cuda.synchronize()
+        barrier()
+        sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    total_ms = max_over_ranks(sum(step_ms))
+    st = ll.ll_status(h)
+    if st != ll.LL_OK:
+        raise SystemExit(f"device status after timing: {ll.status_string(st)}")
+    value = world * args.steps * flops / (total_ms * 1e-3) / 1e12
+
+    # ------------------------------------------- end to end (host buffers)
+    xh = inp.x.contiguous().pin_memory()
+    yh = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            ll.ll_forward_host(h, xh.data_ptr(), yh.data_ptr(), w.M, stream)
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(e2e_steps):
+            flush.zero_()
+            e0[i].record(stream)
+            ll.ll_forward_host(h, xh.data_ptr(), yh.data_ptr(), w.M, stream)
+            e1[i].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)))
+    e2e_value = world * e2e_steps * flops / (e2e_ms * 1e-3) / 1e12
+
+    # ------------------------------------ per-kernel times (profiling mode)
+    ll.ll_set_profiling(h, True)
+    prof_steps = max(3, min(args.steps, 50))
+    per_kernel = {}
+    with torch.cuda.stream(stream):
+        for i in range(prof_steps + 2):
+            flush.zero_()
+            ll.ll_forward(h, x, y, w.M, stream)
+            if i >= 2:
+                for name, ms in ll.ll_kernel_times(h):
+                    per_kernel.setdefault(name, []).append(ms)
+    ll.ll_set_profiling(h, False)
+    torch.cuda.synchronize()
+    kernel_ms = {k: statistics.mean(v) for k, v in per_kernel.items()}
+    dom = max(kernel_ms, key=kernel_ms.get)
+    dom_ms = max_over_ranks(kernel_ms[dom])
+
+    peaks, peak_src = load_peaks()
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if main_flops / main_bytes >= ridge:
+        ach = main_flops / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "peak_source": f"bf16 burst, of {peak_src}"}
+    else:
+        ach = main_bytes / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "peak_source": f"copy bandwidth, of {peak_src}"}
+    roof["kernel"] = dom
+    roof["kernel_ms"] = dom_ms
+    roof["traffic"] = recorded_traffic(dom, w.name)
+    roof["kernel_ms_all"] = kernel_ms
+
+    line = {
+        "metric": "ll_forward TFLOP/s (algorithmic)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "r": w.r,
+                   "scale_mode": "per_row" if w.scale_mode == SCALE_PER_ROW else "per_tensor",
+                   "global_tokens": world * w.M, "parallelism": f"token-sharded replicas x{world}",
+                   "l2": "flushed between steps (256 MiB write, outside the step events)",
+                   "hbm_gbs_algorithmic": world * args.steps * bytes_ / (total_ms * 1e-3) / 1e9},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": 2 * w.M * w.K,
+                "d2h_bytes_per_step": 2 * w.M * w.N, "steps": e2e_steps,
+                "api": "ll_forward_host (pinned host buffers)"},
+        "gpu_launches": launches,
+        "roofline": roof,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    layer.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

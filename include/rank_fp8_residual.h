@@ -63,8 +63,11 @@ enum {
   LL_ERR_DEVICE_TIMEOUT = 7  /* a device-side wait ran past its limit */
 };
 
-/* Kernel variants for ll_set_variant. */
-enum { LL_VARIANT_AUTO = 0, LL_VARIANT_TC = 1 };
+/* Kernel variants for ll_set_variant: AUTO picks by M (SMALL for M <= 128,
+ * TC above); TC is the fused 128x256-tile kernel with the folded low-rank
+ * factor; SMALL is the 128x128-tile kernel with separate residual and
+ * low-rank accumulators. */
+enum { LL_VARIANT_AUTO = 0, LL_VARIANT_TC = 1, LL_VARIANT_SMALL = 2 };
 
 /* Create a layer with N output features, K input features and rank r on
  * the current CUDA device.  Requires N >= 1 and N % 8 == 0, K >= 16 and
@@ -80,9 +83,11 @@ ll_handle ll_create(int N, int K, int r, int scale_mode);
  * the layer's scale_mode; bias: bf16 [N] or NULL.  All non-NULL pointers
  * must be 16-byte aligned device pointers except scale and bias (4- and
  * 2-byte aligned).  The rank is zero-padded internally to a multiple of
- * 64 (exact).  Returns LL_ERR_NAN_CODE if any Q code is 0x7F or 0xFF;
- * LL_ERR_INVALID_ARG for null/misaligned/non-device pointers or a
- * non-finite scale. */
+ * 32 (exact).  The call also prepares A / scale as a bf16 pair for the
+ * fused large-M kernel.  Returns LL_ERR_NAN_CODE if any Q code is 0x7F or
+ * 0xFF; LL_ERR_INVALID_ARG for null/misaligned/non-device pointers or a
+ * non-finite scale; LL_ERR_UNSUPPORTED if some nonzero |A[n,j] / scale[n]|
+ * lies outside [2^-100, 2^100] (rows with scale 0 count as scale 1). */
 int ll_set_weights(ll_handle h, const void *A, const void *B, const void *Q, const float *scale,
                    const void *bias);
 
@@ -130,6 +135,21 @@ const char *ll_status_string(int code);
 
 /* Number of kernels the last ll_forward on this handle launched. */
 int ll_last_launch_count(ll_handle h);
+
+/* Profiling mode (enable != 0): every later ll_forward records CUDA events
+ * on its stream around each kernel it launches, and launches them without
+ * programmatic overlap so each duration is that kernel's alone.  All work
+ * is still done.  Off by default. */
+int ll_set_profiling(ll_handle h, int enable);
+
+/* Device durations in milliseconds of the kernels the last profiled
+ * ll_forward launched, in launch order, written to ms[0 .. n).  Waits for
+ * the events.  Returns the number of kernels (may exceed n), or -1 if the
+ * last forward was not profiled. */
+int ll_kernel_times(ll_handle h, float *ms, int n);
+
+/* Name of the i-th kernel of the last ll_forward (static string), or NULL. */
+const char *ll_kernel_name(ll_handle h, int i);
 
 #ifdef __cplusplus
 }

@@ -5,7 +5,7 @@ step of the forward runs in the library's CUDA kernels.  Functions keep the
 C names and accept either raw integers (device addresses, stream handles)
 or torch tensors / streams, from which they take ``data_ptr()`` and
 ``cuda_stream``.  There is no CPU fallback: importing raises if the shared
-library has not been built (``python -m rank_fp8_residual_b200.build``).
+library has not been built (``python rank_fp8_residual_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -28,6 +28,7 @@ LL_ERR_DEVICE_TIMEOUT = 7
 
 LL_VARIANT_AUTO = 0
 LL_VARIANT_TC = 1
+LL_VARIANT_SMALL = 2
 
 # Every symbol the header declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -44,6 +45,9 @@ _SIGNATURES = {
     "ll_last_error": (ctypes.c_int, []),
     "ll_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ll_last_launch_count": (ctypes.c_int, [_P]),
+    "ll_set_profiling": (ctypes.c_int, [_P, ctypes.c_int]),
+    "ll_kernel_times": (ctypes.c_int, [_P, _P, ctypes.c_int]),
+    "ll_kernel_name": (ctypes.c_char_p, [_P, ctypes.c_int]),
 }
 
 
@@ -56,7 +60,7 @@ class LLError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m rank_fp8_residual_b200.build`")
+            f"{LIB_PATH} is missing: build it with `python rank_fp8_residual_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():
         fn = getattr(lib, name)
@@ -146,6 +150,21 @@ def ll_destroy(h: int) -> None:
 
 def ll_last_launch_count(h: int) -> int:
     return _lib.ll_last_launch_count(h)
+
+
+def ll_set_profiling(h: int, enable: bool) -> None:
+    rc = _lib.ll_set_profiling(h, int(bool(enable)))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_set_profiling")
+
+
+def ll_kernel_times(h: int):
+    """[(kernel name, device ms)] of the last profiled forward."""
+    buf = (ctypes.c_float * 8)()
+    n = _lib.ll_kernel_times(h, ctypes.cast(buf, ctypes.c_void_p), 8)
+    if n < 0:
+        raise LLError(LL_ERR_CUDA, "ll_kernel_times")
+    return [(_lib.ll_kernel_name(h, i).decode(), float(buf[i])) for i in range(min(n, 8))]
 
 
 class LiteLinearLayer:

@@ -1,8 +1,9 @@
 """Build step of the CUDA library: compiles csrc/ for sm_100a into
 rank_fp8_residual_b200/librank_fp8_residual_b200.so (in-tree).
 
-Run as ``python -m rank_fp8_residual_b200.build`` (add ``-v`` for the
-ptxas resource report).  nvcc cross-compiles without a GPU.
+Run as ``python rank_fp8_residual_b200/build.py`` (add ``-v`` for the
+ptxas resource report); it is a standalone file so that it runs without
+importing the package.  nvcc cross-compiles without a GPU.
 """
 from __future__ import annotations
 

@@ -1,7 +1,7 @@
 // Host side of the C ABI declared in include/rank_fp8_residual.h:
 // argument validation, handle-owned device copies of the factors, TMA
 // tensor-map construction, workspace management and the kernel chain of
-// one forward (see ll_kernels.cuh).
+// one forward (kernels in ll_kernels.cuh and ll_tc.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -15,6 +15,7 @@
 
 #include "../../include/rank_fp8_residual.h"
 #include "ll_kernels.cuh"
+#include "ll_tc.cuh"
 
 namespace {
 
@@ -43,9 +44,9 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor [rows, cols] of `elem` bytes per element, row pitch
-// `pitch_bytes`; box = {box_cols, box_rows}.
-bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, uint64_t rows, uint64_t cols,
+// 2-D row-major tensor [rows, cols], row pitch `pitch_bytes`; box =
+// {box_cols, box_rows}.  Elements outside the tensor load as zeros.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
               uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -53,11 +54,12 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  (void)elem;
   CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
 bool is_device_ptr(const void* p) {
   cudaPointerAttributes a;
@@ -70,20 +72,32 @@ bool is_device_ptr(const void* p) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+int next_pow2_ge32(int v) {
+  int p = 32;
+  while (p < v) p <<= 1;
+  return p;
+}
+
 }  // namespace
 
 struct ll_layer {
-  int N = 0, K = 0, r = 0, r_pad = 0, scale_mode = 0;
+  int N = 0, K = 0, r = 0, r_pad = 0, klr = 64, scale_mode = 0;
   int device = 0, num_sms = 0;
   bool ready = false;
   bool has_bias = false;
-  uint8_t* Q = nullptr;
-  uint16_t* A = nullptr;  // [N, r_pad]
-  uint16_t* B = nullptr;  // [r_pad, K]
-  float* scale = nullptr; // [N]
-  uint16_t* bias = nullptr;
-  int* status = nullptr;  // device status word
-  int* nanflag = nullptr;
+  // factors (device, handle-owned)
+  uint8_t* Q = nullptr;       // [N, K] e4m3fn codes as given
+  uint8_t* Qf = nullptr;      // rows with zero scale cleared (== Q when no scale is zero)
+  uint16_t* A = nullptr;      // [N, r_pad] bf16, zero-padded
+  uint16_t* Ahi = nullptr;    // [N, r_pad] bf16 of A / s_eff
+  uint16_t* Alo = nullptr;    // [N, r_pad] bf16 of A / s_eff - Ahi
+  uint16_t* B = nullptr;      // [r_pad, K] bf16, zero-padded
+  float* scale = nullptr;     // [N] scale as given (broadcast for per-tensor)
+  float* scale_eff = nullptr; // [N] scale, 1 where the scale is zero
+  uint16_t* bias = nullptr;   // [N]
+  int* status = nullptr;      // device status word
+  int* flags = nullptr;       // [2] set-time scan flags
+  int* sched = nullptr;       // [2] tile scheduler of the fused kernel
   // workspace for t
   int ws_M = 0;
   uint16_t* t_hi = nullptr;
@@ -95,29 +109,41 @@ struct ll_layer {
   void* dy = nullptr;
   size_t dx_bytes = 0, dy_bytes = 0;
   // weight tensor maps
-  CUtensorMap tm_q, tm_a, tm_b;
-  int rc = 64;
+  CUtensorMap tm_q, tm_qf, tm_a, tm_ahi, tm_alo, tm_b;
+  int b_box = 0;
   // per-call cache
   const void* c_x = nullptr;
-  void* c_y = nullptr;
+  void* c_yptr = nullptr;
   int c_M = -1;
-  CUtensorMap c_tm_x, c_tm_y, c_tm_thi, c_tm_tlo;
+  CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256;
   int variant = LL_VARIANT_AUTO;
   int withhold = 0;
   uint64_t timeout_ns = 2000000000ull;
   int last_launches = 0;
+  // profiling
+  int profiling = 0;
+  int prof_valid = 0;
+  cudaEvent_t ev[8] = {};
+  const char* names[8] = {};
 };
 
 namespace {
 
 void free_layer_mem(ll_layer* h) {
+  for (cudaEvent_t& e : h->ev)
+    if (e) cudaEventDestroy(e);
+  if (h->Qf && h->Qf != h->Q) cudaFree(h->Qf);
   cudaFree(h->Q);
   cudaFree(h->A);
+  cudaFree(h->Ahi);
+  cudaFree(h->Alo);
   cudaFree(h->B);
   cudaFree(h->scale);
+  cudaFree(h->scale_eff);
   cudaFree(h->bias);
   cudaFree(h->status);
-  cudaFree(h->nanflag);
+  cudaFree(h->flags);
+  cudaFree(h->sched);
   cudaFree(h->t_hi);
   cudaFree(h->t_lo);
   cudaFree(h->part);
@@ -133,6 +159,9 @@ int set_smem_attrs_once() {
     if (cudaFuncSetAttribute(llk::ll_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::main_smem_bytes()) != cudaSuccess)
       rc = 1;
+    if (cudaFuncSetAttribute(llk::ll_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::tc_smem_bytes()) != cudaSuccess)
+      rc = 1;
     if (cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::lr_smem_bytes(256)) != cudaSuccess)
       rc = 1;
@@ -140,12 +169,13 @@ int set_smem_attrs_once() {
   return rc;
 }
 
-// Grow the t workspace to hold `M` rows (stream-ordered).
+// Grow the t workspace to hold `M` rows and the split partials to
+// `part_need` bytes (stream-ordered).
 int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
   if (h->r_pad == 0) return LL_OK;
   if (M > h->ws_M) {
     int newM = std::max(M, h->ws_M * 3 / 2);
-    newM = (newM + 127) / 128 * 128;
+    newM = (newM + 255) / 256 * 256;
     uint16_t *th = nullptr, *tl = nullptr;
     const size_t bytes = static_cast<size_t>(newM) * h->r_pad * sizeof(uint16_t);
     if (cudaMallocAsync(reinterpret_cast<void**>(&th), bytes, st) != cudaSuccess ||
@@ -159,7 +189,7 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
     h->t_hi = th;
     h->t_lo = tl;
     h->ws_M = newM;
-    h->c_M = -1;  // invalidate maps over t
+    h->c_M = -1;  // maps over t must be rebuilt
   }
   if (part_need > h->part_bytes) {
     float* pp = nullptr;
@@ -175,29 +205,41 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
   return LL_OK;
 }
 
+bool use_tc(const ll_layer* h, int M) {
+  if (h->variant == LL_VARIANT_TC) return true;
+  if (h->variant == LL_VARIANT_SMALL) return false;
+  return M > 128;
+}
+
 struct LrPlan {
-  int rc, ksplit, kb_per_split, m_tiles, r_chunks;
+  int rc;            // column block of t per CTA (B box height)
+  int tmem_cols;     // power of two >= rc
+  int ksplit, kb_per_split, m_tiles, r_chunks;
 };
 
 LrPlan plan_lowrank(const ll_layer* h, int M) {
   LrPlan p{};
   const int nK = (h->K + llk::kBK - 1) / llk::kBK;
   p.m_tiles = (M + 127) / 128;
-  if (h->r_pad == 0) {  // no low-rank term: nothing to plan
-    p.rc = 64;
+  if (h->r_pad == 0) {
+    p.rc = 32;
+    p.tmem_cols = 32;
     p.ksplit = 1;
     p.kb_per_split = nK;
     p.r_chunks = 0;
     return p;
   }
-  // Column block of t per CTA: the widest of 256/128/64 that divides r_pad
-  // (TMEM allocations are powers of two); 128 when the token count alone
-  // cannot occupy half the GPU, so that more CTAs share the read of B.
-  p.rc = (h->r_pad % 256 == 0) ? 256 : (h->r_pad % 128 == 0) ? 128 : 64;
-  if (p.rc == 256 && p.m_tiles * (h->r_pad / 128) <= h->num_sms / 2) p.rc = 128;
-  p.r_chunks = h->r_pad / p.rc;
+  p.rc = std::min(h->r_pad, 256);
+  const bool fused_large = use_tc(h, M);
+  // Few token tiles: narrower column blocks so more CTAs share the read of B.
+  if (!fused_large && p.rc > 128 && p.m_tiles * ((h->r_pad + 127) / 128) <= h->num_sms / 2) p.rc = 128;
+  p.r_chunks = (h->r_pad + p.rc - 1) / p.rc;
+  p.tmem_cols = next_pow2_ge32(p.rc);
   const int ctas = p.m_tiles * p.r_chunks;
-  int ks = std::max(1, h->num_sms / ctas);
+  // With the fused large-M kernel the down-projection runs beside it on a
+  // quarter of the SMs; the small-M kernel waits for it, so it takes all.
+  const int budget = fused_large ? std::max(1, h->num_sms / 4) : h->num_sms;
+  int ks = std::max(1, budget / ctas);
   ks = std::min(ks, nK);
   p.kb_per_split = (nK + ks - 1) / ks;
   p.ksplit = (nK + p.kb_per_split - 1) / p.kb_per_split;
@@ -210,24 +252,25 @@ size_t part_bytes_for(const ll_layer* h, int M) {
 }
 
 bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
-  if (h->c_x == x && h->c_y == y && h->c_M == M) return true;
+  if (h->c_x == x && h->c_yptr == y && h->c_M == M) return true;
   using namespace llk;
-  if (!make_map(&h->c_tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->K, 2ull * h->K, kBK, 128,
-                CU_TENSOR_MAP_SWIZZLE_128B))
-    return false;
-  if (!make_map(&h->c_tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->N, 2ull * h->N, 32, 32,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
-    return false;
+  bool ok = true;
+  ok &= make_map(&h->c_x128, x, kBF16, M, h->K, 2ull * h->K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&h->c_x256, x, kBF16, M, h->K, 2ull * h->K, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&h->c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (h->r_pad > 0) {
-    if (!make_map(&h->c_tm_thi, h->t_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->r_pad, 2ull * h->r_pad, kBK,
-                  128, CU_TENSOR_MAP_SWIZZLE_128B))
-      return false;
-    if (!make_map(&h->c_tm_tlo, h->t_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, h->r_pad, 2ull * h->r_pad, kBK,
-                  128, CU_TENSOR_MAP_SWIZZLE_128B))
-      return false;
+    const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    ok &= make_map(&h->c_thi128, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->c_tlo128, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->c_thi256, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
+    ok &= make_map(&h->c_tlo256, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
+  }
+  if (!ok) {
+    h->c_M = -1;
+    return false;
   }
   h->c_x = x;
-  h->c_y = y;
+  h->c_yptr = y;
   h->c_M = M;
   return true;
 }
@@ -235,23 +278,30 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
 int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) {
   using namespace llk;
   h->last_launches = 0;
+  const bool tc = use_tc(h, M);
   const LrPlan lp = plan_lowrank(h, M);
-  int rc = ensure_workspace(h, M, st, lp.ksplit > 1 ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0);
+  int rc = ensure_workspace(h, M, st,
+                            lp.ksplit > 1 ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0);
   if (rc != LL_OK) return rc;
   if (!build_call_maps(h, x, y, M)) return LL_ERR_CUDA;
   const Watch watch{h->status, h->timeout_ns};
   int launches = 0;
+  const bool prof = h->profiling != 0;
+  h->prof_valid = 0;
+  if (prof) {
+    for (cudaEvent_t& e : h->ev)
+      if (!e && cudaEventCreate(&e) != cudaSuccess) return LL_ERR_CUDA;
+    cudaEventRecord(h->ev[0], st);
+  }
 
   if (h->r_pad > 0) {
-    LrDownParams lpp;
-    lpp.tm_x = h->c_tm_x;
-    // B map for the chosen column block height.
-    if (lp.rc != h->rc) {
-      if (!make_map(&h->tm_b, h->B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->r_pad, h->K, 2ull * h->K, kBK, lp.rc,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
+    if (lp.rc != h->b_box) {
+      if (!make_map(&h->tm_b, h->B, kBF16, h->r_pad, h->K, 2ull * h->K, kBK, lp.rc, CU_TENSOR_MAP_SWIZZLE_128B))
         return LL_ERR_CUDA;
-      h->rc = lp.rc;
+      h->b_box = lp.rc;
     }
+    LrDownParams lpp;
+    lpp.tm_x = h->c_x128;
     lpp.tm_b = h->tm_b;
     lpp.t_hi = h->t_hi;
     lpp.t_lo = h->t_lo;
@@ -260,56 +310,95 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     lpp.K = h->K;
     lpp.r_pad = h->r_pad;
     lpp.rc = lp.rc;
+    lpp.tmem_cols = lp.tmem_cols;
     lpp.ksplit = lp.ksplit;
     lpp.kb_per_split = lp.kb_per_split;
     lpp.watch = watch;
     dim3 grid(lp.m_tiles, lp.r_chunks, lp.ksplit);
     ll_lrdown_kernel<<<grid, kLrThreads, lr_smem_bytes(lp.rc), st>>>(lpp);
-    ++launches;
+    h->names[launches++] = "ll_lrdown_kernel";
+    if (prof) cudaEventRecord(h->ev[launches], st);
     if (lp.ksplit > 1) {
       const size_t total4 = static_cast<size_t>(M) * h->r_pad / 4;
       int blocks = static_cast<int>(std::min<size_t>((total4 + 255) / 256, static_cast<size_t>(h->num_sms) * 4));
       ll_lrsplit_kernel<<<blocks, 256, 0, st>>>(h->part, h->t_hi, h->t_lo, M, h->r_pad, lp.ksplit);
-      ++launches;
+      h->names[launches++] = "ll_lrsplit_kernel";
+      if (prof) cudaEventRecord(h->ev[launches], st);
     }
     if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
   }
 
-  MainParams mp;
-  mp.tm_x = h->c_tm_x;
-  mp.tm_q = h->tm_q;
-  mp.tm_a = h->tm_a;
-  mp.tm_thi = h->c_tm_thi;
-  mp.tm_tlo = h->c_tm_tlo;
-  mp.tm_y = h->c_tm_y;
-  mp.scale = h->scale;
-  mp.bias = h->has_bias ? h->bias : nullptr;
-  mp.M = M;
-  mp.N = h->N;
-  mp.K = h->K;
-  mp.r_pad = h->r_pad;
-  mp.n_ftiles = (h->N + 127) / 128;
-  mp.n_ttiles = (M + 127) / 128;
-  mp.lr_from_primary = h->r_pad > 0 ? 1 : 0;
-  mp.withhold = h->withhold;
-  mp.watch = watch;
-  const int tiles = mp.n_ftiles * mp.n_ttiles;
-
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(std::min(tiles, h->num_sms));
-  cfg.blockDim = dim3(kMainThreads);
-  cfg.dynamicSmemBytes = main_smem_bytes();
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = h->r_pad > 0 ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, ll_main_kernel, mp) != cudaSuccess) {
+  cfg.numAttrs = (h->r_pad > 0 && !prof) ? 1 : 0;
+  cudaError_t err;
+  if (tc) {
+    TcParams tp;
+    tp.tm_x = h->c_x256;
+    tp.tm_q = h->tm_qf;
+    tp.tm_ahi = h->tm_ahi;
+    tp.tm_alo = h->tm_alo;
+    tp.tm_thi = h->c_thi256;
+    tp.tm_tlo = h->c_tlo256;
+    tp.tm_y = h->c_y;
+    tp.scale = h->scale_eff;
+    tp.bias = h->has_bias ? h->bias : nullptr;
+    tp.sched = h->sched;
+    tp.M = M;
+    tp.N = h->N;
+    tp.K = h->K;
+    tp.r_pad = h->r_pad;
+    tp.klr = h->klr;
+    tp.n_ftiles = (h->N + 127) / 128;
+    tp.n_ttiles = (M + kTcBT - 1) / kTcBT;
+    tp.lr_from_primary = h->r_pad > 0 ? 1 : 0;
+    tp.withhold = h->withhold;
+    tp.watch = watch;
+    const int tiles = tp.n_ftiles * tp.n_ttiles;
+    cfg.gridDim = dim3(std::min(tiles, h->num_sms));
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = tc_smem_bytes();
+    err = cudaLaunchKernelEx(&cfg, ll_tc_kernel, tp);
+    h->names[launches] = "ll_tc_kernel";
+  } else {
+    MainParams mp;
+    mp.tm_x = h->c_x128;
+    mp.tm_q = h->tm_q;
+    mp.tm_a = h->tm_a;
+    mp.tm_thi = h->c_thi128;
+    mp.tm_tlo = h->c_tlo128;
+    mp.tm_y = h->c_y;
+    mp.scale = h->scale;
+    mp.bias = h->has_bias ? h->bias : nullptr;
+    mp.M = M;
+    mp.N = h->N;
+    mp.K = h->K;
+    mp.r_pad = h->r_pad;
+    mp.n_ftiles = (h->N + 127) / 128;
+    mp.n_ttiles = (M + 127) / 128;
+    mp.lr_from_primary = h->r_pad > 0 ? 1 : 0;
+    mp.withhold = h->withhold;
+    mp.watch = watch;
+    const int tiles = mp.n_ftiles * mp.n_ttiles;
+    cfg.gridDim = dim3(std::min(tiles, h->num_sms));
+    cfg.blockDim = dim3(kMainThreads);
+    cfg.dynamicSmemBytes = main_smem_bytes();
+    err = cudaLaunchKernelEx(&cfg, ll_main_kernel, mp);
+    h->names[launches] = "ll_main_kernel";
+  }
+  if (err != cudaSuccess) {
     cudaGetLastError();
     return LL_ERR_CUDA;
   }
   ++launches;
+  if (prof) {
+    cudaEventRecord(h->ev[launches], st);
+    h->prof_valid = 1;
+  }
   h->last_launches = launches;
   return LL_OK;
 }
@@ -369,18 +458,24 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
   h->N = N;
   h->K = K;
   h->r = r;
-  h->r_pad = (r + 63) / 64 * 64;
+  h->r_pad = (r + 31) / 32 * 32;
+  h->klr = (h->r_pad % 64 == 0) ? 64 : 32;
   h->scale_mode = scale_mode;
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
   bool ok = true;
+  const size_t nrp = static_cast<size_t>(N) * h->r_pad;
   ok &= cudaMalloc(&h->Q, static_cast<size_t>(N) * K) == cudaSuccess;
   ok &= cudaMalloc(&h->scale, sizeof(float) * N) == cudaSuccess;
+  ok &= cudaMalloc(&h->scale_eff, sizeof(float) * N) == cudaSuccess;
   ok &= cudaMalloc(&h->bias, sizeof(uint16_t) * N) == cudaSuccess;
   ok &= cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
-  ok &= cudaMalloc(&h->nanflag, sizeof(int)) == cudaSuccess;
+  ok &= cudaMalloc(&h->flags, 2 * sizeof(int)) == cudaSuccess;
+  ok &= cudaMalloc(&h->sched, 2 * sizeof(int)) == cudaSuccess;
   if (h->r_pad > 0) {
-    ok &= cudaMalloc(&h->A, sizeof(uint16_t) * N * static_cast<size_t>(h->r_pad)) == cudaSuccess;
+    ok &= cudaMalloc(&h->A, sizeof(uint16_t) * nrp) == cudaSuccess;
+    ok &= cudaMalloc(&h->Ahi, sizeof(uint16_t) * nrp) == cudaSuccess;
+    ok &= cudaMalloc(&h->Alo, sizeof(uint16_t) * nrp) == cudaSuccess;
     ok &= cudaMalloc(&h->B, sizeof(uint16_t) * static_cast<size_t>(h->r_pad) * K) == cudaSuccess;
   }
   if (!ok) {
@@ -390,17 +485,20 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
     fail(LL_ERR_OOM);
     return nullptr;
   }
+  h->Qf = h->Q;
   cudaMemset(h->status, 0, sizeof(int));
+  cudaMemset(h->sched, 0, 2 * sizeof(int));
   using namespace llk;
-  ok &= make_map(&h->tm_q, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  ok &= make_map(&h->tm_q, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  h->tm_qf = h->tm_q;
   if (h->r_pad > 0) {
-    ok &= make_map(&h->tm_a, h->A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, h->r_pad, 2ull * h->r_pad, kBK, 128,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
-    h->rc = std::min(h->r_pad, 256);
-    ok &= make_map(&h->tm_b, h->B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->r_pad, K, 2ull * K, kBK, h->rc,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
+    const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    ok &= make_map(&h->tm_a, h->A, kBF16, N, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->tm_ahi, h->Ahi, kBF16, N, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
+    ok &= make_map(&h->tm_alo, h->Alo, kBF16, N, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
   }
-  if (!ok) {
+  if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
     free_layer_mem(h);
     delete h;
     fail(LL_ERR_CUDA);
@@ -421,7 +519,6 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
       (h->r > 0 && (!aligned(A, 2) || !aligned(B, 2))))
     return fail(LL_ERR_INVALID_ARG);
   const int N = h->N, K = h->K, r = h->r, rp = h->r_pad;
-  // scale must be finite
   const int ns = h->scale_mode == LL_SCALE_PER_ROW ? N : 1;
   std::vector<float> hs(ns);
   if (cudaMemcpy(hs.data(), scale, sizeof(float) * ns, cudaMemcpyDeviceToHost) != cudaSuccess) {
@@ -430,32 +527,52 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
   }
   for (float v : hs)
     if (!std::isfinite(v)) return fail(LL_ERR_INVALID_ARG);
-  // NaN-code scan of the residual (before touching the handle's copy).
-  if (cudaMemset(h->nanflag, 0, sizeof(int)) != cudaSuccess) return fail(LL_ERR_CUDA);
+  std::vector<float> full(N), eff(N);
+  bool any_zero = false;
+  for (int n = 0; n < N; ++n) {
+    full[n] = hs[h->scale_mode == LL_SCALE_PER_ROW ? n : 0];
+    eff[n] = full[n] == 0.f ? 1.f : full[n];
+    any_zero |= full[n] == 0.f;
+  }
+  // NaN-code scan of the residual before anything of the handle changes.
+  if (cudaMemset(h->flags, 0, 2 * sizeof(int)) != cudaSuccess) return fail(LL_ERR_CUDA);
   const size_t nq = static_cast<size_t>(N) * K;
   llk::ll_nan_scan_kernel<<<std::max(1, std::min(h->num_sms * 8, static_cast<int>((nq / 16 + 255) / 256))), 256>>>(
-      static_cast<const uint8_t*>(Q), nq, h->nanflag);
+      static_cast<const uint8_t*>(Q), nq, h->flags);
   int flag = 0;
   if (cudaGetLastError() != cudaSuccess ||
-      cudaMemcpy(&flag, h->nanflag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+      cudaMemcpy(&flag, h->flags, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
     cudaGetLastError();
     return fail(LL_ERR_CUDA);
   }
   if (flag) return fail(LL_ERR_NAN_CODE);
+  h->ready = false;
   bool ok = true;
   ok &= cudaMemcpy(h->Q, Q, nq, cudaMemcpyDeviceToDevice) == cudaSuccess;
-  if (h->scale_mode == LL_SCALE_PER_ROW) {
-    ok &= cudaMemcpy(h->scale, scale, sizeof(float) * N, cudaMemcpyDeviceToDevice) == cudaSuccess;
-  } else {
-    std::vector<float> full(N, hs[0]);
-    ok &= cudaMemcpy(h->scale, full.data(), sizeof(float) * N, cudaMemcpyHostToDevice) == cudaSuccess;
-  }
+  ok &= cudaMemcpy(h->scale, full.data(), sizeof(float) * N, cudaMemcpyHostToDevice) == cudaSuccess;
+  ok &= cudaMemcpy(h->scale_eff, eff.data(), sizeof(float) * N, cudaMemcpyHostToDevice) == cudaSuccess;
   if (bias) {
     ok &= cudaMemcpy(h->bias, bias, sizeof(uint16_t) * N, cudaMemcpyDeviceToDevice) == cudaSuccess;
   } else {
     ok &= cudaMemset(h->bias, 0, sizeof(uint16_t) * N) == cudaSuccess;
   }
   h->has_bias = bias != nullptr;
+  // Residual used by the fused large-M kernel: rows with zero scale cleared.
+  if (any_zero) {
+    if (h->Qf == h->Q) {
+      ok &= cudaMalloc(&h->Qf, nq) == cudaSuccess;
+      ok &= make_map(&h->tm_qf, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, llk::kBK, 128,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+    }
+    if (ok) {
+      llk::ll_zero_rows_kernel<<<h->num_sms * 8, 256>>>(h->Q, h->scale, h->Qf, N, K);
+      ok &= cudaGetLastError() == cudaSuccess;
+    }
+  } else if (h->Qf != h->Q) {
+    cudaFree(h->Qf);
+    h->Qf = h->Q;
+    h->tm_qf = h->tm_q;
+  }
   if (rp > 0) {
     ok &= cudaMemset(h->A, 0, sizeof(uint16_t) * N * static_cast<size_t>(rp)) == cudaSuccess;
     ok &= cudaMemset(h->B, 0, sizeof(uint16_t) * static_cast<size_t>(rp) * K) == cudaSuccess;
@@ -463,13 +580,23 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
                        cudaMemcpyDeviceToDevice) == cudaSuccess;
     ok &= cudaMemcpy(h->B, B, sizeof(uint16_t) * static_cast<size_t>(r) * K, cudaMemcpyDeviceToDevice) ==
           cudaSuccess;
+    if (ok) {
+      llk::ll_fold_prep_kernel<<<h->num_sms * 8, 256>>>(h->A, h->scale_eff, h->Ahi, h->Alo, N, rp,
+                                                         h->flags + 1);
+      ok &= cudaGetLastError() == cudaSuccess;
+    }
   }
   ok &= cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
-    h->ready = false;
     return fail(LL_ERR_CUDA);
   }
+  int range_flag = 0;
+  if (rp > 0 && cudaMemcpy(&range_flag, h->flags + 1, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  if (range_flag) return fail(LL_ERR_UNSUPPORTED);  // |A / scale| outside [2^-100, 2^100]
   h->ready = true;
   return LL_OK;
 }
@@ -543,7 +670,8 @@ int ll_reserve(ll_handle h, int max_M) {
 
 int ll_set_variant(ll_handle h, int variant) {
   g_last_error = LL_OK;
-  if (!h || (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC)) return fail(LL_ERR_INVALID_ARG);
+  if (!h || (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC && variant != LL_VARIANT_SMALL))
+    return fail(LL_ERR_INVALID_ARG);
   h->variant = variant;
   return LL_OK;
 }
@@ -558,7 +686,9 @@ int ll_status(ll_handle h) {
     return fail(LL_ERR_CUDA);
   }
   if (v != 0) {
+    // A kernel gave up part-way: clear the status and the tile scheduler.
     cudaMemset(h->status, 0, sizeof(int));
+    cudaMemset(h->sched, 0, 2 * sizeof(int));
     cudaDeviceSynchronize();
     return LL_ERR_DEVICE_TIMEOUT;
   }
@@ -574,6 +704,38 @@ int ll_set_debug(ll_handle h, int withhold_producer, uint64_t timeout_ns) {
 }
 
 int ll_last_launch_count(ll_handle h) { return h ? h->last_launches : 0; }
+
+int ll_set_profiling(ll_handle h, int enable) {
+  g_last_error = LL_OK;
+  if (!h) return fail(LL_ERR_INVALID_ARG);
+  h->profiling = enable ? 1 : 0;
+  return LL_OK;
+}
+
+int ll_kernel_times(ll_handle h, float* ms, int n) {
+  g_last_error = LL_OK;
+  if (!h || !h->prof_valid) return -1;
+  if (cudaEventSynchronize(h->ev[h->last_launches]) != cudaSuccess) {
+    cudaGetLastError();
+    fail(LL_ERR_CUDA);
+    return -1;
+  }
+  for (int i = 0; i < h->last_launches && i < n; ++i) {
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]) != cudaSuccess) {
+      cudaGetLastError();
+      fail(LL_ERR_CUDA);
+      return -1;
+    }
+    if (ms) ms[i] = t;
+  }
+  return h->last_launches;
+}
+
+const char* ll_kernel_name(ll_handle h, int i) {
+  if (!h || i < 0 || i >= h->last_launches) return nullptr;
+  return h->names[i];
+}
 
 void ll_destroy(ll_handle h) {
   if (!h) return;

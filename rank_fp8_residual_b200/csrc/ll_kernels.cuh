@@ -73,7 +73,8 @@ struct LrDownParams {
   uint16_t* t_lo;    // [M, r_pad]
   float* part;       // [ksplit, M, r_pad] fp32 (ksplit > 1)
   int M, K, r_pad;
-  int rc;            // rows of B (= columns of t) per CTA: 64, 128 or 256
+  int rc;            // box height of B = column block of t per CTA (<= 256)
+  int tmem_cols;     // power of two >= rc
   int ksplit;        // number of K splits (gridDim.z)
   int kb_per_split;  // 64-wide K steps per split
   Watch watch;
@@ -98,11 +99,12 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128;
   const int j0 = blockIdx.y * p.rc;
+  const int wcols = min(p.rc, p.r_pad - j0);  // columns of t this CTA owns (multiple of 32)
   const int kz = blockIdx.z;
   const int nK = (p.K + kBK - 1) / kBK;
   const int kb_begin = kz * p.kb_per_split;
   const int kb_end = min(nK, kb_begin + p.kb_per_split);
-  const int ncols = p.rc;  // TMEM columns = fp32 accumulator width
+  const int ncols = p.tmem_cols;
 
   if (threadIdx.x == 0) {
     pdl_launch_dependents();
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, p.rc);
+      const uint32_t idesc = idesc_bf16(128, wcols);
       int s = 0;
       uint32_t ph = 0;
       bool first = true;
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
     if (__all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.watch, kErrTimeoutEpilogue))) {
       tc_fence_after();
       const bool empty_range = kb_end <= kb_begin;
-      for (int c = 0; c < p.rc; c += 32) {
+      for (int c = 0; c < wcols; c += 32) {
         uint32_t v[32];
         tmem_ld32_wait(tbase + ((32u * q) << 16) + c, v);
         if (m < p.M) {
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kMainThreads, 1) ll_main_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = p.n_ftiles * p.n_ttiles;
   const int nK = (p.K + kBK - 1) / kBK;
-  const int nR = p.r_pad / kBK;
+  const int nR = (p.r_pad + kBK - 1) / kBK;  // columns past r_pad load as zeros
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }

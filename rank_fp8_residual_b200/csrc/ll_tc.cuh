@@ -1,0 +1,434 @@
+// Large-M fused kernel (sm_100a) of the LiteLinear forward
+//
+//     y = (x B^T) A^T + scale * (x Q^T) + bias            (LiteLinear README,
+//                                                          introduction)
+//
+// evaluated per output row n as
+//
+//     y[m, n] = s[n] * ( sum_k Q[n,k] x[m,k] + sum_j A'[n,j] t[m,j] ) + bias[n]
+//
+// with t = x B^T (from ll_lrdown_kernel, carried as bf16 t_hi + t_lo) and
+// A' = A / s[n] carried as bf16 A'_hi + A'_lo (prepared once when the
+// weights are set).  Multiplying out, s*A'*t = A*t, so the single fp32
+// accumulator holds both terms and the epilogue applies s[n] and the bias
+// once.  The low-rank product uses three bf16 MMAs per K step
+// (A'_hi t_hi + A'_hi t_lo + A'_lo t_hi); the dropped A'_lo t_lo term and
+// the two pair splittings leave a relative error of order 2^-16 on the
+// low-rank term.  Rows with s[n] == 0 use s = 1 and an all-zero residual row
+// (exact, since 0 * (x Q^T) = 0).
+//
+// Tile: 128 output features (MMA M, TMEM lanes) x up to 256 tokens (MMA N,
+// TMEM columns).  Q is the MMA A operand: eight converter warps widen the
+// e4m3fn codes exactly to bf16 and store them into TMEM stages; x is the B
+// operand, staged by TMA.  Persistent CTAs take tiles from a device-wide
+// counter in a grouped raster order (8 token tiles per group) so that the
+// tiles in flight share their x and Q slabs in L2.
+//
+// Warp roles (14 warps): 0 TMA producer + tile scheduler, 1 MMA issuer
+// (also allocates TMEM), 2-9 converters (lane quadrant w%4, K half
+// (w-2)/4), 10-13 epilogue (lane quadrant w%4).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+#include "ll_kernels.cuh"
+#include "ptx.cuh"
+
+namespace llk {
+
+struct TcParams {
+  CUtensorMap tm_x;    // bf16 [M, K]       box {64, 256},  128B swizzle
+  CUtensorMap tm_q;    // u8   [N, K]       box {64, 128},   64B swizzle
+  CUtensorMap tm_ahi;  // bf16 [N, r_pad]   box {klr, 128}, 128B (klr 64) / 64B (klr 32) swizzle
+  CUtensorMap tm_alo;  // bf16 [N, r_pad]
+  CUtensorMap tm_thi;  // bf16 [M, r_pad]   box {klr, 256}
+  CUtensorMap tm_tlo;  // bf16 [M, r_pad]
+  CUtensorMap tm_y;    // bf16 [M, N]       box {32, 32},    no swizzle
+  const float* scale;    // effective per-row scale [N]
+  const uint16_t* bias;  // [N] bf16 bits, or nullptr
+  int* sched;            // [2]: tile counter, finished-CTA counter (0 between launches)
+  int M, N, K, r_pad, klr;
+  int n_ftiles, n_ttiles;
+  int lr_from_primary;
+  int withhold;
+  Watch watch;
+};
+
+constexpr int kTcThreads = 448;
+constexpr int kTcBT = 256;                  // tokens per tile
+constexpr int kTcSX = 4;                    // 32 KB slots: x chunks, A'/t chunks
+constexpr int kTcSQ = 6;                    // 8 KB slots: Q chunks
+constexpr int kTcNA = 8;                    // widened-Q stages in TMEM (32 columns each)
+constexpr int kTcXSlot = kTcBT * kBK * 2;   // 32768
+constexpr int kTcQSlot = 128 * kBK;         // 8192
+constexpr int kTcEpi = 4 * 2 * 32 * 32 * 2; // 4 warps x 2 buffers x (32 tokens x 32 features) bf16
+constexpr int kTcGroup = 8;                 // token tiles per raster group
+constexpr int kTcConvWarps = 8;
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcTileRing = 2;
+constexpr int kTcColA = 256;                // TMEM column of the first widened-Q stage
+
+__host__ __device__ constexpr int tc_smem_bytes() {
+  return kTcSX * kTcXSlot + kTcSQ * kTcQSlot + kTcEpi + 1024 + 512;
+}
+
+__device__ __forceinline__ void tc_tile_coords(int T, int n_ftiles, int n_ttiles, int& f0, int& t0) {
+  const int per_group = kTcGroup * n_ftiles;
+  const int g = T / per_group;
+  const int first_tt = g * kTcGroup;
+  const int gsize = min(kTcGroup, n_ttiles - first_tt);
+  const int idx = T - g * per_group;
+  f0 = (idx / gsize) * 128;
+  t0 = (first_tt + idx % gsize) * kTcBT;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sx = smem;
+  uint8_t* sq = sx + kTcSX * kTcXSlot;
+  uint8_t* se = sq + kTcSQ * kTcQSlot;
+  uint64_t* x_full = reinterpret_cast<uint64_t*>(se + kTcEpi);
+  uint64_t* x_empty = x_full + kTcSX;
+  uint64_t* q_full = x_empty + kTcSX;
+  uint64_t* q_empty = q_full + kTcSQ;
+  uint64_t* a_full = q_empty + kTcSQ;
+  uint64_t* a_empty = a_full + kTcNA;
+  uint64_t* acc_full = a_empty + kTcNA;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* tile_full = acc_empty + 1;
+  uint64_t* tile_empty = tile_full + kTcTileRing;
+  uint64_t* drain = tile_empty + kTcTileRing;
+  int* tile_slot = reinterpret_cast<int*>(drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_slot + kTcTileRing);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = p.n_ftiles * p.n_ttiles;
+  const int nK = (p.K + kBK - 1) / kBK;
+  const int nR = p.r_pad / p.klr;
+  const int klr = p.klr;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcSX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
+    for (int s = 0; s < kTcSQ; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], kTcConvWarps); }
+    for (int s = 0; s < kTcNA; ++s) { mbar_init(&a_full[s], kTcConvWarps); mbar_init(&a_empty[s], 1); }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kTcEpiWarps);
+    for (int s = 0; s < kTcTileRing; ++s) {
+      mbar_init(&tile_full[s], 1);
+      mbar_init(&tile_empty[s], 1 + kTcConvWarps + kTcEpiWarps);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tm_x);
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_y);
+    if (nR > 0) {
+      tma_prefetch_desc(&p.tm_ahi);
+      tma_prefetch_desc(&p.tm_alo);
+      tma_prefetch_desc(&p.tm_thi);
+      tma_prefetch_desc(&p.tm_tlo);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------- TMA + tile scheduler
+    if (lane == 0) {
+      int xi = 0, qi = 0, ti = 0;
+      uint32_t xph = 0, qph = 0, tph = 0;
+      long long nx = 0, nq = 0;
+      bool ok = true, waited_primary = false;
+      int T = blockIdx.x;
+      const uint32_t a_bytes = 128u * klr * 2u;
+      const uint32_t t_bytes = static_cast<uint32_t>(kTcBT) * klr * 2u;
+      for (;;) {
+        if (!mbar_wait(&tile_empty[ti], tph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+        const bool live = T < n_tiles;
+        *reinterpret_cast<volatile int*>(&tile_slot[ti]) = live ? T : -1;
+        mbar_arrive(&tile_full[ti]);
+        if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
+        if (!live) break;
+        if (p.withhold) { ok = false; break; }  // debug: no loads, the consumers time out
+        const int next = static_cast<int>(gridDim.x) + atomicAdd(&p.sched[0], 1);
+        int f0, t0;
+        tc_tile_coords(T, p.n_ftiles, p.n_ttiles, f0, t0);
+        for (int kb = 0; kb < nK && ok; ++kb) {
+          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&x_full[xi], kTcXSlot);
+          tma_load_2d(sx + xi * kTcXSlot, &p.tm_x, &x_full[xi], kb * kBK, t0);
+          ++nx;
+          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          if (!mbar_wait(&q_empty[qi], qph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[qi], kTcQSlot);
+          tma_load_2d(sq + qi * kTcQSlot, &p.tm_q, &q_full[qi], kb * kBK, f0);
+          ++nq;
+          if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
+        }
+        if (ok && nR > 0 && !waited_primary && p.lr_from_primary) {
+          pdl_wait_primary();
+          waited_primary = true;
+        }
+        for (int jb = 0; jb < nR && ok; ++jb) {
+          // slot 1: A'_hi | A'_lo chunk; slot 2: t_hi chunk; slot 3: t_lo chunk
+          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&x_full[xi], 2 * a_bytes);
+          tma_load_2d(sx + xi * kTcXSlot, &p.tm_ahi, &x_full[xi], jb * klr, f0);
+          tma_load_2d(sx + xi * kTcXSlot + a_bytes, &p.tm_alo, &x_full[xi], jb * klr, f0);
+          ++nx;
+          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&x_full[xi], t_bytes);
+          tma_load_2d(sx + xi * kTcXSlot, &p.tm_thi, &x_full[xi], jb * klr, t0);
+          ++nx;
+          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&x_full[xi], t_bytes);
+          tma_load_2d(sx + xi * kTcXSlot, &p.tm_tlo, &x_full[xi], jb * klr, t0);
+          ++nx;
+          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+        }
+        if (!ok) break;
+        T = next;
+      }
+      if (!ok) {
+        for (long long i = (nx > kTcSX ? nx - kTcSX : 0); i < nx; ++i)
+          mbar_wait_drain(&x_full[i % kTcSX], static_cast<uint32_t>((i / kTcSX) & 1), p.watch);
+        for (long long i = (nq > kTcSQ ? nq - kTcSQ : 0); i < nq; ++i)
+          mbar_wait_drain(&q_full[i % kTcSQ], static_cast<uint32_t>((i / kTcSQ) & 1), p.watch);
+      }
+      // The last CTA to finish resets the scheduler for the next launch.
+      __threadfence();
+      if (atomicAdd(&p.sched[1], 1) == static_cast<int>(gridDim.x) - 1) {
+        atomicExch(&p.sched[0], 0);
+        atomicExch(&p.sched[1], 0);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      int xi = 0, ai = 0, ti = 0;
+      uint32_t xph = 0, aph = 0, accph = 0, tph = 0;
+      bool ok = true;
+      const uint32_t a_bytes = 128u * klr * 2u;
+      for (;;) {
+        if (!mbar_wait(&tile_full[ti], tph, p.watch, kErrTimeoutMma)) break;
+        const int T = *reinterpret_cast<volatile int*>(&tile_slot[ti]);
+        mbar_arrive(&tile_empty[ti]);
+        if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
+        if (T < 0) break;
+        int f0, t0;
+        tc_tile_coords(T, p.n_ftiles, p.n_ttiles, f0, t0);
+        const int valid = min(kTcBT, p.M - t0);
+        const uint32_t idesc = idesc_bf16(128, (valid + 15) & ~15);
+        if (!mbar_wait(acc_empty, accph ^ 1, p.watch, kErrTimeoutMma)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < nK; ++kb) {
+          if (!mbar_wait(&a_full[ai], aph, p.watch, kErrTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait(&x_full[xi], xph, p.watch, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sx + xi * kTcXSlot));
+          const uint32_t at = tbase + kTcColA + ai * 32;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_ts(tbase, at + kk * 8, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          tc_commit(&x_empty[xi]);
+          tc_commit(&a_empty[ai]);
+          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          if (++ai == kTcNA) { ai = 0; aph ^= 1; }
+        }
+        for (int jb = 0; jb < nR && ok; ++jb) {
+          int slot[3];
+          for (int w = 0; w < 3; ++w) {
+            if (!mbar_wait(&x_full[xi], xph, p.watch, kErrTimeoutMma)) { ok = false; break; }
+            slot[w] = xi;
+            if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          }
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sx + slot[0] * kTcXSlot);
+          const uint32_t sh = smem_u32(sx + slot[1] * kTcXSlot);
+          const uint32_t sl = smem_u32(sx + slot[2] * kTcXSlot);
+          uint64_t ah, al, th, tl;
+          if (klr == 64) {
+            ah = sdesc_kmajor_sw128(sa); al = sdesc_kmajor_sw128(sa + a_bytes);
+            th = sdesc_kmajor_sw128(sh); tl = sdesc_kmajor_sw128(sl);
+          } else {
+            ah = sdesc_kmajor_sw64(sa); al = sdesc_kmajor_sw64(sa + a_bytes);
+            th = sdesc_kmajor_sw64(sh); tl = sdesc_kmajor_sw64(sl);
+          }
+          for (int kk = 0; kk < klr / 16; ++kk) {
+            mma_ss(tbase, ah + 2 * kk, th + 2 * kk, idesc, 1u);
+            mma_ss(tbase, ah + 2 * kk, tl + 2 * kk, idesc, 1u);
+            mma_ss(tbase, al + 2 * kk, th + 2 * kk, idesc, 1u);
+          }
+          for (int w = 0; w < 3; ++w) tc_commit(&x_empty[slot[w]]);
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        accph ^= 1;
+      }
+      tc_commit(drain);
+      mbar_wait_drain(drain, 0, p.watch);
+    }
+  } else if (warp < 2 + kTcConvWarps) {
+    // ----------------------------------------- e4m3 -> bf16 into TMEM stages
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;           // which 32 of the 64 K columns
+    const int row = 32 * q + lane;              // feature row within the tile
+    const int sw = (row >> 1) & 3;              // 64-byte swizzle phase of the row
+    const uint32_t tl = tbase + ((32u * q) << 16) + kTcColA + 16 * half;
+    int qi = 0, ai = 0, ti = 0;
+    uint32_t qph = 0, aph = 0, tph = 0;
+    bool ok = true;
+    for (;;) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&tile_full[ti], tph, p.watch, kErrTimeoutConvert))) break;
+      const int T = *reinterpret_cast<volatile int*>(&tile_slot[ti]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tile_empty[ti]);
+      if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
+      if (T < 0) break;
+      // Software pipeline: the codes of step kb+1 are read from shared
+      // memory before step kb is stored into TMEM.
+      uint4 v0, v1;
+      {
+        if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qi], qph, p.watch, kErrTimeoutConvert))) break;
+        const uint8_t* rb = sq + qi * kTcQSlot + row * 64;
+        v0 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half) ^ sw));
+        v1 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half + 1) ^ sw));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_empty[qi]);
+        if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
+      }
+      for (int kb = 0; kb < nK; ++kb) {
+        uint32_t w[16];
+        e4m3x4_to_bf16x4(v0.x, w[0], w[1]);
+        e4m3x4_to_bf16x4(v0.y, w[2], w[3]);
+        e4m3x4_to_bf16x4(v0.z, w[4], w[5]);
+        e4m3x4_to_bf16x4(v0.w, w[6], w[7]);
+        e4m3x4_to_bf16x4(v1.x, w[8], w[9]);
+        e4m3x4_to_bf16x4(v1.y, w[10], w[11]);
+        e4m3x4_to_bf16x4(v1.z, w[12], w[13]);
+        e4m3x4_to_bf16x4(v1.w, w[14], w[15]);
+        if (kb + 1 < nK) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qi], qph, p.watch, kErrTimeoutConvert))) {
+            ok = false;
+            break;
+          }
+          const uint8_t* rb = sq + qi * kTcQSlot + row * 64;
+          v0 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half) ^ sw));
+          v1 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half + 1) ^ sw));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&q_empty[qi]);
+          if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[ai], aph ^ 1, p.watch, kErrTimeoutConvert))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(tl + ai * 32, w);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[ai]);
+        if (++ai == kTcNA) { ai = 0; aph ^= 1; }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int frow = 32 * q + lane;
+    const uint32_t tl = tbase + ((32u * q) << 16);
+    uint16_t* stage = reinterpret_cast<uint16_t*>(se + (warp - 2 - kTcConvWarps) * (2 * 32 * 32 * 2));
+    int eb = 0, ti = 0;
+    uint32_t accph = 0, tph = 0;
+    for (;;) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&tile_full[ti], tph, p.watch, kErrTimeoutEpilogue))) break;
+      const int T = *reinterpret_cast<volatile int*>(&tile_slot[ti]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tile_empty[ti]);
+      if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
+      if (T < 0) break;
+      int f0, t0;
+      tc_tile_coords(T, p.n_ftiles, p.n_ttiles, f0, t0);
+      const int valid = min(kTcBT, p.M - t0);
+      const int f = f0 + frow;
+      const float s = f < p.N ? p.scale[f] : 0.f;
+      const float b = (p.bias != nullptr && f < p.N) ? bf16_bits_to_float(p.bias[f]) : 0.f;
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_full, accph, p.watch, kErrTimeoutEpilogue))) break;
+      tc_fence_after();
+      const bool store_rows = f0 + 32 * q < p.N;
+      for (int c = 0; c < valid; c += 32) {
+        uint32_t v[32];
+        tmem_ld32_wait(tl + c, v);
+        if (lane == 0) tma_store_wait_read<1>();
+        __syncwarp();
+        uint16_t* st = stage + eb * (32 * 32);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) st[i * 32 + lane] = to_bf16_bits(fmaf(s, __uint_as_float(v[i]), b));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (store_rows) tma_store_2d(&p.tm_y, st, f0 + 32 * q, t0 + c);
+          tma_store_commit();
+        }
+        eb ^= 1;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      accph ^= 1;
+    }
+    if (lane == 0) tma_store_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// Set-time preparation of the folded low-rank factor: A' = A / s_eff[n]
+// split into a bf16 pair (hi = bf16(A'), lo = bf16(A' - hi)).  Flags any
+// value whose pair would leave bf16's normal range.
+__global__ void ll_fold_prep_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s_eff,
+                                    uint16_t* __restrict__ ahi, uint16_t* __restrict__ alo, int N, int r_pad,
+                                    int* __restrict__ bad) {
+  const size_t total = static_cast<size_t>(N) * r_pad;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(i / r_pad);
+    const float a = bf16_bits_to_float(A[i]);
+    const float ap = a / s_eff[n];
+    const uint16_t h = to_bf16_bits(ap);
+    const uint16_t l = to_bf16_bits(ap - bf16_bits_to_float(h));
+    ahi[i] = h;
+    alo[i] = l;
+    const float m = fabsf(ap);
+    if (!(m <= 0x1p100f) || (m != 0.f && m < 0x1p-100f)) atomicOr(bad, 1);
+  }
+}
+
+// Copy of Q with the rows whose scale is zero cleared.
+__global__ void ll_zero_rows_kernel(const uint8_t* __restrict__ q, const float* __restrict__ scale,
+                                    uint8_t* __restrict__ out, int N, int K) {
+  const size_t total = static_cast<size_t>(N) * K;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(i / K);
+    out[i] = scale[n] == 0.f ? 0 : q[i];
+  }
+}
+
+}  // namespace llk

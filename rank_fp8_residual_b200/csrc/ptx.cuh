@@ -183,6 +183,17 @@ __device__ __forceinline__ void tmem_ld32x2_wait(uint32_t ta, uint32_t (&r)[32],
       : "r"(ta), "r"(tb)
       : "memory");
 }
+// Store 16 consecutive 32-bit TMEM columns of this thread's lane (no wait).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Store 32 consecutive 32-bit TMEM columns of this thread's lane and wait
 // until the stores have been performed.
 __device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -208,6 +219,18 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
   d |= static_cast<uint64_t>(1024u >> 4) << 32;             // stride byte offset: next 8-row group
   d |= static_cast<uint64_t>(1u) << 46;                     // descriptor version (sm_100)
   d |= static_cast<uint64_t>(2u) << 61;                     // layout: 128-byte swizzle
+  return d;
+}
+
+// Same for a K-major tile with the 64-byte swizzle (rows of 64 bytes,
+// 8-row groups 512 bytes apart; base 512-byte aligned).
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw64(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(4u) << 61;  // layout: 64-byte swizzle
   return d;
 }
 

@@ -18,12 +18,17 @@ from llgpu import DeviceLayer, check, run
 pytestmark = pytest.mark.gpu
 
 
-def _full(inp, what):
-    y = run(inp)
-    return check(y, oracle.forward_inputs(inp), what=what)
+VARIANTS = [ll.LL_VARIANT_TC, ll.LL_VARIANT_SMALL]
+VNAME = {ll.LL_VARIANT_TC: "tc", ll.LL_VARIANT_SMALL: "small", ll.LL_VARIANT_AUTO: "auto"}
 
 
-def test_widening_is_exact_for_every_code():
+def _full(inp, what, variant=ll.LL_VARIANT_AUTO):
+    y = run(inp, variant)
+    return check(y, oracle.forward_inputs(inp), what=f"{what} [{VNAME[variant]}]")
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_widening_is_exact_for_every_code(variant):
     """One-hot tokens pick single residual codes: y[m, n] = Q[n, m] exactly.
     Every non-NaN code appears in every K position, so the swizzled shared
     memory reads and the TMEM lane mapping are covered too."""
@@ -35,7 +40,7 @@ def test_widening_is_exact_for_every_code():
     x = torch.eye(M, K, dtype=torch.bfloat16)
     inp = LayerInputs(M, K, N, 0, SCALE_PER_TENSOR, x, None, None, codes,
                       torch.ones(1, dtype=torch.float32), None)
-    y = run(inp).to(torch.float64)
+    y = run(inp, variant).to(torch.float64)
     expect = codes.view(torch.float8_e4m3fn).to(torch.float64).t()  # [M=K, N]
     assert torch.equal(y, expect)
 
@@ -44,38 +49,70 @@ def test_tiny_config():
     _full(WORKLOADS["tiny_m64_k256_n256_r16"].inputs(), "tiny")
 
 
-@pytest.mark.parametrize("M,K,N,r", [(300, 272, 392, 40), (129, 1024, 136, 64), (517, 384, 1000, 200)])
-def test_ragged_multi_tile(M, K, N, r):
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("M,K,N,r", [(300, 272, 392, 40), (129, 1024, 136, 64), (517, 384, 1000, 200),
+                                     (1100, 320, 264, 96)])
+def test_ragged_multi_tile(M, K, N, r, variant):
     inp = make_inputs(M, K, N, r, scale_range=(1e-3, 3e-3), seed=M)
-    _full(inp, f"ragged {M}x{K}x{N} r{r}")
+    _full(inp, f"ragged {M}x{K}x{N} r{r}", variant)
 
 
-def test_rank_zero():
-    _full(make_inputs(200, 256, 256, 0, seed=1), "r=0")
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_rank_zero(variant):
+    _full(make_inputs(600, 256, 256, 0, seed=1), "r=0", variant)
 
 
-def test_residual_zero_is_low_rank_only():
-    _full(make_inputs(200, 256, 256, 32, seed=2, q_zero=True), "Q=0")
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_residual_zero_is_low_rank_only(variant):
+    _full(make_inputs(600, 256, 256, 32, seed=2, q_zero=True), "Q=0", variant)
 
 
-def test_per_tensor_scale_and_no_bias():
-    _full(make_inputs(150, 320, 264, 24, scale_mode=SCALE_PER_TENSOR, bias=False, seed=3),
-          "per-tensor, no bias")
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_per_tensor_scale_and_no_bias(variant):
+    _full(make_inputs(450, 320, 264, 24, scale_mode=SCALE_PER_TENSOR, bias=False, seed=3),
+          "per-tensor, no bias", variant)
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_zero_scale_rows(variant):
+    """Rows with scale 0 keep only their low-rank term and bias."""
+    inp = make_inputs(520, 256, 392, 40, scale_range=(1e-3, 3e-3), seed=4)
+    inp.scale[::7] = 0.0
+    inp.scale[5] = -2e-3  # a negative scale is a valid multiplier
+    _full(inp, "zero-scale rows", variant)
+
+
+def test_scale_far_outside_fold_range_is_rejected():
+    """The fused large-M kernel carries A / scale as a bf16 pair; a scale
+    that would push it past 2^100 is reported instead of losing accuracy."""
+    inp = make_inputs(8, 64, 64, 8, seed=5)
+    inp.scale[3] = 1e-35
+    h = ll.ll_create(64, 64, 8, SCALE_PER_ROW)
+    try:
+        with pytest.raises(ll.LLError) as e:
+            ll.ll_set_weights(h, inp.A.cuda(), inp.B.cuda(), inp.Q.cuda(), inp.scale.cuda(),
+                              inp.bias.cuda())
+        assert e.value.code == ll.LL_ERR_UNSUPPORTED
+    finally:
+        ll.ll_destroy(h)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 31, 64])
-def test_small_token_counts(M):
-    _full(make_inputs(M, 512, 1024, 96, seed=10 + M), f"M={M}")
+def test_small_token_counts(M, variant):
+    _full(make_inputs(M, 512, 1024, 96, seed=10 + M), f"M={M}", variant)
 
 
-@pytest.mark.parametrize("M", [127, 128, 129, 255, 257])
-def test_token_tile_edges(M):
-    _full(make_inputs(M, 128, 256, 16, seed=20 + M), f"M={M}")
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("M", [127, 128, 129, 255, 256, 257, 511, 513])
+def test_token_tile_edges(M, variant):
+    _full(make_inputs(M, 128, 256, 16, seed=20 + M), f"M={M}", variant)
 
 
-@pytest.mark.parametrize("r", [1, 63, 64, 65, 128, 256, 320, 512])
-def test_rank_edges(r):
-    _full(make_inputs(140, 256, 256, r, seed=30 + r), f"r={r}")
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("r", [1, 31, 32, 33, 63, 64, 65, 96, 128, 160, 256, 320, 512])
+def test_rank_edges(r, variant):
+    _full(make_inputs(300, 256, 256, r, seed=30 + r), f"r={r}", variant)
 
 
 def test_attention_projection_full():
@@ -91,7 +128,7 @@ def _sampled_rows(M, n=48):
 
 def _sampled(name):
     inp = WORKLOADS[name].inputs()
-    y = run(inp)
+    y = run(inp, ll.LL_VARIANT_AUTO)
     rows = _sampled_rows(inp.M)
     ref = oracle.forward_inputs(inp, rows=rows)
     return check(y[rows], ref, what=name + " (sampled rows)")
