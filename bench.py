@@ -227,6 +227,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", default="auto", choices=["auto", "tc", "tc_pair", "small"],
+                    help="kernel variant (auto picks by token count)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -257,6 +259,8 @@ def main():
                       inp.Q.to(dev), inp.scale.to(dev),
                       inp.bias.to(dev) if inp.bias is not None else None)
     h = layer.handle
+    ll.ll_set_variant(h, {"auto": ll.LL_VARIANT_AUTO, "tc": ll.LL_VARIANT_TC, "tc_pair": ll.LL_VARIANT_TC_PAIR,
+                          "small": ll.LL_VARIANT_SMALL}[args.variant])
     ll.ll_reserve(h, w.M)
     x = inp.x.to(dev)
     y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
@@ -364,6 +368,7 @@ def main():
         "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "r": w.r,
                    "scale_mode": "per_row" if w.scale_mode == SCALE_PER_ROW else "per_tensor",
                    "global_tokens": world * w.M, "parallelism": f"token-sharded replicas x{world}",
+                   "variant": args.variant,
                    "l2": "flushed between steps (256 MiB write, outside the step events)",
                    "hbm_gbs_algorithmic": world * args.steps * bytes_ / (total_ms * 1e-3) / 1e9},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": 2 * w.M * w.K,

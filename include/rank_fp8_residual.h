@@ -63,11 +63,14 @@ enum {
   LL_ERR_DEVICE_TIMEOUT = 7  /* a device-side wait ran past its limit */
 };
 
-/* Kernel variants for ll_set_variant: AUTO picks by M (SMALL for M <= 128,
- * TC above); TC is the fused 128x256-tile kernel with the folded low-rank
- * factor; SMALL is the 128x128-tile kernel with separate residual and
- * low-rank accumulators. */
-enum { LL_VARIANT_AUTO = 0, LL_VARIANT_TC = 1, LL_VARIANT_SMALL = 2 };
+/* Kernel variants for ll_set_variant.  AUTO: TC for M > 128, SMALL
+ * otherwise.  TC: one-CTA fused kernel, 128 features x 256 tokens per
+ * tile, low-rank factor folded as A / scale (bf16 pair).  TC_PAIR: the
+ * same on CTA pairs (256 features per MMA); slower than TC on every
+ * measured shape, kept selectable for comparison.  SMALL: one-CTA kernel,
+ * 128 x 128 tiles, separate residual and low-rank accumulators.  Every
+ * variant meets the same accuracy bound. */
+enum { LL_VARIANT_AUTO = 0, LL_VARIANT_TC = 1, LL_VARIANT_SMALL = 2, LL_VARIANT_TC_PAIR = 3 };
 
 /* Create a layer with N output features, K input features and rank r on
  * the current CUDA device.  Requires N >= 1 and N % 8 == 0, K >= 16 and

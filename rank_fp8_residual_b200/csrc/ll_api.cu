@@ -16,6 +16,7 @@
 #include "../../include/rank_fp8_residual.h"
 #include "ll_kernels.cuh"
 #include "ll_tc.cuh"
+#include "ll_tc2.cuh"
 
 namespace {
 
@@ -60,6 +61,22 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t
 }
 
 constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+
+// 3-D view {d0, d1, d2} with strides {s1, s2} (bytes) and box {b0, b1, b2}:
+// used to read several 64-wide K chunks of a row-major matrix in one load
+// (d0 = 64 elements of a chunk, d1 = rows, d2 = chunk index).
+bool make_map3(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool is_device_ptr(const void* p) {
   cudaPointerAttributes a;
@@ -115,7 +132,9 @@ struct ll_layer {
   const void* c_x = nullptr;
   void* c_yptr = nullptr;
   int c_M = -1;
-  CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256;
+  CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256, c_thik, c_tlok, c_x3;
+  CUtensorMap tm_q3;  // 3-D view of the (row-cleared) residual, 4 K chunks per box
+  int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
   int variant = LL_VARIANT_AUTO;
   int withhold = 0;
   uint64_t timeout_ns = 2000000000ull;
@@ -162,6 +181,9 @@ int set_smem_attrs_once() {
     if (cudaFuncSetAttribute(llk::ll_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::tc_smem_bytes()) != cudaSuccess)
       rc = 1;
+    if (cudaFuncSetAttribute(llk::ll_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::tc2_smem_bytes()) != cudaSuccess)
+      rc = 1;
     if (cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::lr_smem_bytes(256)) != cudaSuccess)
       rc = 1;
@@ -205,10 +227,18 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
   return LL_OK;
 }
 
-bool use_tc(const ll_layer* h, int M) {
-  if (h->variant == LL_VARIANT_TC) return true;
-  if (h->variant == LL_VARIANT_SMALL) return false;
-  return M > 128;
+enum Path { PATH_SMALL, PATH_TC1, PATH_TC2 };
+
+Path choose_path(const ll_layer* h, int M) {
+  if (h->variant == LL_VARIANT_TC) return PATH_TC1;
+  if (h->variant == LL_VARIANT_TC_PAIR) return PATH_TC2;
+  if (h->variant == LL_VARIANT_SMALL) return PATH_SMALL;
+  return M > 128 ? PATH_TC1 : PATH_SMALL;
+}
+
+// The CTA-pair kernel computes t with the warp-level kernel beside it.
+bool warp_lowrank(const ll_layer* h, int M) {
+  return choose_path(h, M) == PATH_TC2 && h->r_pad > 0 && h->r_pad <= 128;
 }
 
 struct LrPlan {
@@ -230,15 +260,16 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
     return p;
   }
   p.rc = std::min(h->r_pad, 256);
-  const bool fused_large = use_tc(h, M);
+  const Path path = choose_path(h, M);
+  const bool fused_large = path != PATH_SMALL;
   // Few token tiles: narrower column blocks so more CTAs share the read of B.
   if (!fused_large && p.rc > 128 && p.m_tiles * ((h->r_pad + 127) / 128) <= h->num_sms / 2) p.rc = 128;
   p.r_chunks = (h->r_pad + p.rc - 1) / p.rc;
   p.tmem_cols = next_pow2_ge32(p.rc);
   const int ctas = p.m_tiles * p.r_chunks;
-  // With the fused large-M kernel the down-projection runs beside it on a
-  // quarter of the SMs; the small-M kernel waits for it, so it takes all.
-  const int budget = fused_large ? std::max(1, h->num_sms / 4) : h->num_sms;
+  // With the single-CTA fused kernel the down-projection runs beside it on
+  // a quarter of the SMs; the other kernels wait for it, so it takes all.
+  const int budget = path == PATH_TC1 ? std::max(1, h->num_sms / 4) : h->num_sms;
   int ks = std::max(1, budget / ctas);
   ks = std::min(ks, nK);
   p.kb_per_split = (nK + ks - 1) / ks;
@@ -247,6 +278,7 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
 }
 
 size_t part_bytes_for(const ll_layer* h, int M) {
+  if (warp_lowrank(h, M)) return 0;
   const LrPlan p = plan_lowrank(h, M);
   return p.ksplit > 1 ? static_cast<size_t>(p.ksplit) * M * h->r_pad * sizeof(float) : 0;
 }
@@ -258,12 +290,16 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   ok &= make_map(&h->c_x128, x, kBF16, M, h->K, 2ull * h->K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&h->c_x256, x, kBF16, M, h->K, 2ull * h->K, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&h->c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (h->K % 64 == 0) ok &= make_map3(&h->c_x3, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, 128, 2,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (h->r_pad > 0) {
     const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     ok &= make_map(&h->c_thi128, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&h->c_tlo128, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&h->c_thi256, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
     ok &= make_map(&h->c_tlo256, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
+    ok &= make_map(&h->c_thik, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
+    ok &= make_map(&h->c_tlok, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
   }
   if (!ok) {
     h->c_M = -1;
@@ -275,13 +311,38 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   return true;
 }
 
+int launch_warp_lowrank(ll_layer* h, const void* x, int M, cudaStream_t st) {
+  using namespace llk;
+  dim3 grid((M + 15) / 16, h->r_pad / 32);
+  ll_lrdown_warp_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(x), h->B, h->t_hi, h->t_lo, M, h->K,
+                                              h->r_pad);
+  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+int pair_cluster_count(ll_layer* h) {
+  if (h->pair_clusters > 0) return h->pair_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(h->num_sms);
+  cfg.blockDim = dim3(llk::kT2Threads);
+  cfg.dynamicSmemBytes = llk::tc2_smem_bytes();
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, llk::ll_tc2_kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = h->num_sms / 2;
+  }
+  h->pair_clusters = std::min(n, h->num_sms / 2);
+  return h->pair_clusters;
+}
+
 int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) {
   using namespace llk;
   h->last_launches = 0;
-  const bool tc = use_tc(h, M);
+  const Path path = choose_path(h, M);
+  const bool wlr = warp_lowrank(h, M);
   const LrPlan lp = plan_lowrank(h, M);
-  int rc = ensure_workspace(h, M, st,
-                            lp.ksplit > 1 ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0);
+  const size_t part_need =
+      (!wlr && lp.ksplit > 1) ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0;
+  int rc = ensure_workspace(h, M, st, part_need);
   if (rc != LL_OK) return rc;
   if (!build_call_maps(h, x, y, M)) return LL_ERR_CUDA;
   const Watch watch{h->status, h->timeout_ns};
@@ -294,7 +355,12 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     cudaEventRecord(h->ev[0], st);
   }
 
-  if (h->r_pad > 0) {
+  if (wlr) {
+    rc = launch_warp_lowrank(h, x, M, st);
+    if (rc != LL_OK) return rc;
+    h->names[launches++] = "ll_lrdown_warp_kernel";
+    if (prof) cudaEventRecord(h->ev[launches], st);
+  } else if (h->r_pad > 0) {
     if (lp.rc != h->b_box) {
       if (!make_map(&h->tm_b, h->B, kBF16, h->r_pad, h->K, 2ull * h->K, kBK, lp.rc, CU_TENSOR_MAP_SWIZZLE_128B))
         return LL_ERR_CUDA;
@@ -328,15 +394,51 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
   }
 
+  // Programmatic overlap with the kernel that produces t, where the main
+  // kernel's schedule tolerates SMs that start late.
+  const bool overlap = h->r_pad > 0 && !prof && (path != PATH_TC2 || wlr);
   cudaLaunchConfig_t cfg = {};
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = (h->r_pad > 0 && !prof) ? 1 : 0;
+  cfg.numAttrs = overlap ? 1 : 0;
   cudaError_t err;
-  if (tc) {
+  if (path == PATH_TC2) {
+    Tc2Params tp;
+    tp.dims3 = h->K % 64 == 0 ? 1 : 0;
+    tp.tm_x = tp.dims3 ? h->c_x3 : h->c_x128;
+    tp.tm_q = tp.dims3 ? h->tm_q3 : h->tm_qf;
+    tp.xc = tp.dims3 ? 2 : 1;
+    tp.qc = tp.dims3 ? 4 : 1;
+    tp.tm_ahi = h->tm_ahi;
+    tp.tm_alo = h->tm_alo;
+    tp.tm_thi = h->c_thik;
+    tp.tm_tlo = h->c_tlok;
+    tp.tm_y = h->c_y;
+    tp.scale = h->scale_eff;
+    tp.bias = h->has_bias ? h->bias : nullptr;
+    tp.M = M;
+    tp.N = h->N;
+    tp.K = h->K;
+    tp.r_pad = h->r_pad;
+    tp.klr = h->klr;
+    tp.n_fpairs = (h->N + 255) / 256;
+    tp.m32 = (M + 31) / 32 * 32;
+    const long long units = static_cast<long long>(tp.n_fpairs) * tp.m32;
+    const int max_clusters = pair_cluster_count(h);
+    const int clusters = static_cast<int>(std::max<long long>(1, std::min<long long>(max_clusters, (units + 255) / 256)));
+    tp.seg = static_cast<int>(((units + clusters - 1) / clusters + 31) / 32 * 32);
+    tp.lr_from_primary = overlap ? 1 : 0;
+    tp.withhold = h->withhold;
+    tp.watch = watch;
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(kT2Threads);
+    cfg.dynamicSmemBytes = tc2_smem_bytes();
+    err = cudaLaunchKernelEx(&cfg, ll_tc2_kernel, tp);
+    h->names[launches] = "ll_tc2_kernel";
+  } else if (path == PATH_TC1) {
     TcParams tp;
     tp.tm_x = h->c_x256;
     tp.tm_q = h->tm_qf;
@@ -355,7 +457,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     tp.klr = h->klr;
     tp.n_ftiles = (h->N + 127) / 128;
     tp.n_ttiles = (M + kTcBT - 1) / kTcBT;
-    tp.lr_from_primary = h->r_pad > 0 ? 1 : 0;
+    tp.lr_from_primary = overlap ? 1 : 0;
     tp.withhold = h->withhold;
     tp.watch = watch;
     const int tiles = tp.n_ftiles * tp.n_ttiles;
@@ -380,7 +482,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     mp.r_pad = h->r_pad;
     mp.n_ftiles = (h->N + 127) / 128;
     mp.n_ttiles = (M + 127) / 128;
-    mp.lr_from_primary = h->r_pad > 0 ? 1 : 0;
+    mp.lr_from_primary = overlap ? 1 : 0;
     mp.withhold = h->withhold;
     mp.watch = watch;
     const int tiles = mp.n_ftiles * mp.n_ttiles;
@@ -491,6 +593,9 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
   using namespace llk;
   ok &= make_map(&h->tm_q, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
   h->tm_qf = h->tm_q;
+  if (K % 64 == 0)
+    ok &= make_map3(&h->tm_q3, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
+                    CU_TENSOR_MAP_SWIZZLE_64B);
   if (h->r_pad > 0) {
     const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     ok &= make_map(&h->tm_a, h->A, kBF16, N, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -563,6 +668,9 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
       ok &= cudaMalloc(&h->Qf, nq) == cudaSuccess;
       ok &= make_map(&h->tm_qf, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, llk::kBK, 128,
                      CU_TENSOR_MAP_SWIZZLE_64B);
+      if (K % 64 == 0)
+        ok &= make_map3(&h->tm_q3, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
     }
     if (ok) {
       llk::ll_zero_rows_kernel<<<h->num_sms * 8, 256>>>(h->Q, h->scale, h->Qf, N, K);
@@ -572,6 +680,9 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
     cudaFree(h->Qf);
     h->Qf = h->Q;
     h->tm_qf = h->tm_q;
+    if (K % 64 == 0)
+      ok &= make_map3(&h->tm_q3, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (rp > 0) {
     ok &= cudaMemset(h->A, 0, sizeof(uint16_t) * N * static_cast<size_t>(rp)) == cudaSuccess;
@@ -670,7 +781,8 @@ int ll_reserve(ll_handle h, int max_M) {
 
 int ll_set_variant(ll_handle h, int variant) {
   g_last_error = LL_OK;
-  if (!h || (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC && variant != LL_VARIANT_SMALL))
+  if (!h || (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC && variant != LL_VARIANT_SMALL &&
+             variant != LL_VARIANT_TC_PAIR))
     return fail(LL_ERR_INVALID_ARG);
   h->variant = variant;
   return LL_OK;

@@ -18,8 +18,9 @@ from llgpu import DeviceLayer, check, run
 pytestmark = pytest.mark.gpu
 
 
-VARIANTS = [ll.LL_VARIANT_TC, ll.LL_VARIANT_SMALL]
-VNAME = {ll.LL_VARIANT_TC: "tc", ll.LL_VARIANT_SMALL: "small", ll.LL_VARIANT_AUTO: "auto"}
+VARIANTS = [ll.LL_VARIANT_TC, ll.LL_VARIANT_SMALL, ll.LL_VARIANT_TC_PAIR]
+VNAME = {ll.LL_VARIANT_TC: "tc", ll.LL_VARIANT_SMALL: "small", ll.LL_VARIANT_AUTO: "auto",
+         ll.LL_VARIANT_TC_PAIR: "tc-pair"}
 
 
 def _full(inp, what, variant=ll.LL_VARIANT_AUTO):
