@@ -60,7 +60,8 @@ enum {
   LL_ERR_NAN_CODE = 4,       /* Q holds an e4m3fn NaN code (0x7F or 0xFF) */
   LL_ERR_OOM = 5,            /* device allocation failed */
   LL_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
-  LL_ERR_DEVICE_TIMEOUT = 7  /* a device-side wait ran past its limit */
+  LL_ERR_DEVICE_TIMEOUT = 7, /* a device-side wait ran past its limit */
+  LL_ERR_SCRATCH_LIMIT = 8   /* request too large for ll_forward_noalloc's scratch */
 };
 
 /* Kernel variants for ll_set_variant.  AUTO: TC for M > 128, SMALL
@@ -153,6 +154,68 @@ int ll_kernel_times(ll_handle h, float *ms, int n);
 
 /* Name of the i-th kernel of the last ll_forward (static string), or NULL. */
 const char *ll_kernel_name(ll_handle h, int i);
+
+/* ---------------------------------------------------------------------
+ * ll_forward_noalloc: the forward without any device allocation.
+ *
+ * The paper has no counterpart to this call; it serves callers that may
+ * not allocate device memory at all.  Examples: a host framework whose
+ * caching allocator already holds the GPU's memory (an outside cudaMalloc
+ * fails, or fragments that pool behind its back), a plug-in whose host
+ * only lets it use buffers the host hands over, and a latency-critical
+ * loop where cudaMalloc / cudaFree would stall on device-wide
+ * synchronisation.  Such a caller cannot use ll_create (it copies the
+ * factors into library-owned memory) or ll_forward (it grows a workspace
+ * on demand).  This call takes no handle: the caller passes every input
+ * and the output, and the intermediate t = x B^T (bf16 hi + lo), its
+ * split-K partial sums, a device status word and, for a per-tensor scale,
+ * the scale broadcast to N rows live in one static device array of
+ * LL_NOALLOC_SCRATCH_BYTES.  Every GPU on which the library's device code
+ * is loaded holds that array until the process exits.
+ *
+ * y is the forward of ll_forward with the SMALL variant (residual and
+ * low-rank terms in separate accumulators, A used as given) and meets the
+ * same accuracy bound.  Arguments are laid out as described at the top of
+ * this header: x bf16 [M, K], A bf16 [N, r] and B bf16 [r, K] (both NULL
+ * when r == 0), Q e4m3fn codes [N, K], scale fp32 [N] (LL_SCALE_PER_ROW) or
+ * [1] (LL_SCALE_PER_TENSOR), bias bf16 [N] or NULL, y bf16 [M, N]; all
+ * device pointers of the current device; x, y, A, B and Q 16-byte
+ * aligned, scale 4-byte, bias 2-byte; y must not overlap x.  Shapes follow
+ * ll_create (N % 8 == 0, K % 16 == 0, K >= 16, 0 <= r <= 512) and, since
+ * A is read in place, r % 8 == 0.  M == 0 is a no-op.
+ *
+ * Limit: with r32 = r rounded up to a multiple of 32, the call needs
+ *     256 + 4 * M * r32 bytes  (+ 4 * N rounded up to 256 for a per-tensor
+ *     scale), at most LL_NOALLOC_SCRATCH_BYTES.
+ * A larger request returns LL_ERR_SCRATCH_LIMIT and launches nothing
+ * (e.g. r = 512 allows M up to 8191, r = 64 up to 65535).  Split-K
+ * partials only use what is left over; when little is, the down-projection
+ * runs with fewer splits.
+ *
+ * Not checked here: the weights are read as given on every call, with no
+ * scan for NaN codes or non-finite scales (ll_set_weights does those
+ * checks); a Q code 0x7F or 0xFF gives meaningless values.
+ *
+ * Shared scratch: every call on a device uses the same array, and the
+ * array keeps the last call's contents.  Each call clears the status word
+ * and fully rewrites t before reading it.  Calls whose kernels overlap on
+ * the GPU (issued on two streams without ordering, or from two host
+ * threads) race on the array and give wrong results: order them on one
+ * stream or with events.
+ *
+ * Set-up: the first call on each device (made with that device current)
+ * looks up the array's device address and sets kernel attributes; make
+ * that first call before any stream capture.
+ *
+ * Errors: LL_ERR_INVALID_ARG for bad shapes, modes, null / misaligned /
+ * non-device pointers or overlap; LL_ERR_UNSUPPORTED for r % 8 != 0;
+ * LL_ERR_SCRATCH_LIMIT as above; LL_ERR_CUDA when a launch fails.  A
+ * device-side wait that runs past its limit (2 s) ends the kernels early
+ * and leaves y incomplete; this call has no way to report that
+ * afterwards. */
+#define LL_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int ll_forward_noalloc(const void *x, const void *A, const void *B, const void *Q, const float *scale,
+                       int scale_mode, const void *bias, void *y, int M, int N, int K, int r, void *stream);
 
 #ifdef __cplusplus
 }

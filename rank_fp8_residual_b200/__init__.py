@@ -25,6 +25,10 @@ LL_ERR_NAN_CODE = 4
 LL_ERR_OOM = 5
 LL_ERR_CUDA = 6
 LL_ERR_DEVICE_TIMEOUT = 7
+LL_ERR_SCRATCH_LIMIT = 8
+
+# Size of the static device scratch used by ll_forward_noalloc.
+LL_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 LL_VARIANT_AUTO = 0
 LL_VARIANT_TC = 1
@@ -49,6 +53,8 @@ _SIGNATURES = {
     "ll_set_profiling": (ctypes.c_int, [_P, ctypes.c_int]),
     "ll_kernel_times": (ctypes.c_int, [_P, _P, ctypes.c_int]),
     "ll_kernel_name": (ctypes.c_char_p, [_P, ctypes.c_int]),
+    "ll_forward_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, _P]),
 }
 
 
@@ -166,6 +172,19 @@ def ll_kernel_times(h: int):
     if n < 0:
         raise LLError(LL_ERR_CUDA, "ll_kernel_times")
     return [(_lib.ll_kernel_name(h, i).decode(), float(buf[i])) for i in range(min(n, 8))]
+
+
+def ll_forward_noalloc(x, A, B, Q, scale, scale_mode: int, bias, y, M: int, N: int, K: int, r: int,
+                       stream=None) -> None:
+    """Forward for callers that may not allocate device memory: no handle,
+    every buffer the caller's, scratch in the library's static device array
+    (LL_NOALLOC_SCRATCH_BYTES per GPU).  Calls on one device must not
+    overlap on the GPU; the first call on a device should precede any
+    stream capture."""
+    rc = _lib.ll_forward_noalloc(_addr(x), _addr(A), _addr(B), _addr(Q), _addr(scale), int(scale_mode), _addr(bias),
+                                 _addr(y), int(M), int(N), int(K), int(r), _stream(stream))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_forward_noalloc")
 
 
 class LiteLinearLayer:

@@ -519,6 +519,7 @@ const char* ll_status_string(int code) {
     case LL_ERR_OOM: return "device allocation failed";
     case LL_ERR_CUDA: return "CUDA call failed";
     case LL_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case LL_ERR_SCRATCH_LIMIT: return "request exceeds the static scratch of ll_forward_noalloc";
     default: return "unknown status";
   }
 }
@@ -858,3 +859,230 @@ void ll_destroy(ll_handle h) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// ll_forward_noalloc: the SMALL kernel chain (down-projection, optional
+// split-K reduction, fused residual + low-rank kernel) with every piece of
+// scratch in one static device array, for callers that may not allocate.
+// Only additions here: the handle-based forward above is untouched.
+
+// File-scope scratch, one instance per GPU on which this module is loaded.
+// Host code must not use this name as an address (on the host it is a
+// stand-in object); the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+
+struct NoAllocDevice {
+  std::once_flag once;
+  int rc = LL_ERR_CUDA;
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
+  int num_sms = 0;
+};
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+// Once per device, with that device current: the scratch address, the SM
+// count and the kernels' shared-memory limits.
+NoAllocDevice* noalloc_setup(int dev, int* rc) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) {
+    *rc = LL_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  NoAllocDevice& d = g_noalloc_dev[dev];
+  std::call_once(d.once, [&d, dev] {
+    void* p = nullptr;
+    int sms = 0;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0 ||
+        cudaFuncSetAttribute(llk::ll_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::main_smem_bytes()) != cudaSuccess ||
+        cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::lr_smem_bytes(256)) != cudaSuccess) {
+      cudaGetLastError();
+      d.rc = LL_ERR_CUDA;
+      return;
+    }
+    d.scratch = static_cast<unsigned char*>(p);
+    d.num_sms = sms;
+    d.rc = LL_OK;
+  });
+  *rc = d.rc;
+  return d.rc == LL_OK ? &d : nullptr;
+}
+
+// A per-tensor scale, repeated for each of the N output features.
+__global__ void ll_noalloc_scale_kernel(const float* __restrict__ s, float* __restrict__ out, int N) {
+  const float v = s[0];
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) out[i] = v;
+}
+
+size_t round_up256(size_t v) { return (v + 255) / 256 * 256; }
+
+int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, const float* scale, int scale_mode,
+                    const void* bias, void* y, int M, int N, int K, int r, cudaStream_t st) {
+  using namespace llk;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
+  int rc = LL_OK;
+  NoAllocDevice* d = noalloc_setup(dev, &rc);
+  if (!d) return rc;
+
+  // Scratch layout: status word | broadcast scale (per-tensor only) |
+  // t_hi [M, r_pad] | t_lo [M, r_pad] | split-K partials (what is left).
+  const int r_pad = (r + 31) / 32 * 32;
+  const size_t t_bytes = static_cast<size_t>(M) * r_pad * sizeof(uint16_t);
+  size_t off = 256;
+  const size_t scale_off = off;
+  if (scale_mode == LL_SCALE_PER_TENSOR) off += round_up256(static_cast<size_t>(N) * sizeof(float));
+  const size_t thi_off = off;
+  const size_t tlo_off = thi_off + t_bytes;
+  const size_t part_off = tlo_off + t_bytes;  // 64-byte aligned: t rows are 64-byte multiples
+  if (part_off > LL_NOALLOC_SCRATCH_BYTES) return LL_ERR_SCRATCH_LIMIT;
+
+  unsigned char* base = d->scratch;
+  int* status = reinterpret_cast<int*>(base);
+  const float* scale_n = scale;
+  if (scale_mode == LL_SCALE_PER_TENSOR) scale_n = reinterpret_cast<float*>(base + scale_off);
+  uint16_t* t_hi = reinterpret_cast<uint16_t*>(base + thi_off);
+  uint16_t* t_lo = reinterpret_cast<uint16_t*>(base + tlo_off);
+  float* part = reinterpret_cast<float*>(base + part_off);
+
+  // Down-projection plan of the SMALL path, with the number of K splits
+  // cut to what the remaining scratch holds.
+  ll_layer view;
+  view.N = N;
+  view.K = K;
+  view.r = r;
+  view.r_pad = r_pad;
+  view.num_sms = d->num_sms;
+  view.variant = LL_VARIANT_SMALL;
+  LrPlan lp = plan_lowrank(&view, M);
+  if (r_pad > 0 && lp.ksplit > 1) {
+    const size_t per_split = static_cast<size_t>(M) * r_pad * sizeof(float);
+    const size_t fit = (LL_NOALLOC_SCRATCH_BYTES - part_off) / per_split;
+    if (fit < static_cast<size_t>(lp.ksplit)) {
+      const int nK = (K + kBK - 1) / kBK;
+      const int ks = fit < 2 ? 1 : static_cast<int>(fit);
+      lp.kb_per_split = (nK + ks - 1) / ks;
+      lp.ksplit = (nK + lp.kb_per_split - 1) / lp.kb_per_split;
+    }
+  }
+
+  // Tensor maps over the caller's buffers; rank columns / rows past r read
+  // as zeros (TMA fill), which stands in for the zero padding to r_pad.
+  CUtensorMap tm_x, tm_q, tm_a, tm_b, tm_thi, tm_tlo, tm_y;
+  bool ok = make_map(&tm_x, x, kBF16, M, K, 2ull * K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&tm_q, Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  ok &= make_map(&tm_y, y, kBF16, M, N, 2ull * N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (r_pad > 0) {
+    ok &= make_map(&tm_a, A, kBF16, N, r, 2ull * r, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&tm_b, B, kBF16, r, K, 2ull * K, kBK, lp.rc, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&tm_thi, t_hi, kBF16, M, r_pad, 2ull * r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&tm_tlo, t_lo, kBF16, M, r_pad, 2ull * r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    tm_a = tm_x;  // unused when r_pad == 0
+    tm_thi = tm_x;
+    tm_tlo = tm_x;
+  }
+  if (!ok) return LL_ERR_CUDA;
+
+  const Watch watch{status, 2000000000ull};
+  if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
+  if (scale_mode == LL_SCALE_PER_TENSOR) {
+    const int blocks = std::max(1, std::min((N + 255) / 256, 4 * d->num_sms));
+    ll_noalloc_scale_kernel<<<blocks, 256, 0, st>>>(scale, const_cast<float*>(scale_n), N);
+  }
+  if (r_pad > 0) {
+    LrDownParams lpp;
+    lpp.tm_x = tm_x;
+    lpp.tm_b = tm_b;
+    lpp.t_hi = t_hi;
+    lpp.t_lo = t_lo;
+    lpp.part = part;
+    lpp.M = M;
+    lpp.K = K;
+    lpp.r_pad = r_pad;
+    lpp.rc = lp.rc;
+    lpp.tmem_cols = lp.tmem_cols;
+    lpp.ksplit = lp.ksplit;
+    lpp.kb_per_split = lp.kb_per_split;
+    lpp.watch = watch;
+    dim3 grid(lp.m_tiles, lp.r_chunks, lp.ksplit);
+    ll_lrdown_kernel<<<grid, kLrThreads, lr_smem_bytes(lp.rc), st>>>(lpp);
+    if (lp.ksplit > 1) {
+      const size_t total4 = static_cast<size_t>(M) * r_pad / 4;
+      const int blocks =
+          static_cast<int>(std::min<size_t>((total4 + 255) / 256, static_cast<size_t>(d->num_sms) * 4));
+      ll_lrsplit_kernel<<<blocks, 256, 0, st>>>(part, t_hi, t_lo, M, r_pad, lp.ksplit);
+    }
+  }
+  if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
+
+  MainParams mp;
+  mp.tm_x = tm_x;
+  mp.tm_q = tm_q;
+  mp.tm_a = tm_a;
+  mp.tm_thi = tm_thi;
+  mp.tm_tlo = tm_tlo;
+  mp.tm_y = tm_y;
+  mp.scale = scale_n;
+  mp.bias = static_cast<const uint16_t*>(bias);
+  mp.M = M;
+  mp.N = N;
+  mp.K = K;
+  mp.r_pad = r_pad;
+  mp.n_ftiles = (N + 127) / 128;
+  mp.n_ttiles = (M + 127) / 128;
+  mp.lr_from_primary = r_pad > 0 ? 1 : 0;
+  mp.withhold = 0;
+  mp.watch = watch;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = r_pad > 0 ? 1 : 0;
+  cfg.gridDim = dim3(std::min(mp.n_ftiles * mp.n_ttiles, d->num_sms));
+  cfg.blockDim = dim3(kMainThreads);
+  cfg.dynamicSmemBytes = main_smem_bytes();
+  if (cudaLaunchKernelEx(&cfg, ll_main_kernel, mp) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
+  return LL_OK;
+}
+
+}  // namespace
+
+extern "C" int ll_forward_noalloc(const void* x, const void* A, const void* B, const void* Q, const float* scale,
+                                  int scale_mode, const void* bias, void* y, int M, int N, int K, int r,
+                                  void* stream) {
+  g_last_error = LL_OK;
+  if (M < 0 || N < 1 || K < 16 || r < 0 || r > 512 || (N % 8) != 0 || (K % 16) != 0 ||
+      (scale_mode != LL_SCALE_PER_TENSOR && scale_mode != LL_SCALE_PER_ROW))
+    return fail(LL_ERR_INVALID_ARG);
+  if (M == 0) return LL_OK;
+  if (r % 8 != 0) return fail(LL_ERR_UNSUPPORTED);
+  if (!x || !y || !Q || !scale || (r > 0 && (!A || !B))) return fail(LL_ERR_INVALID_ARG);
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(Q, 16) || !aligned(scale, 4) || (bias && !aligned(bias, 2)) ||
+      (r > 0 && (!aligned(A, 16) || !aligned(B, 16))))
+    return fail(LL_ERR_INVALID_ARG);
+  const char* xb = static_cast<const char*>(x);
+  const char* yb = static_cast<const char*>(y);
+  const size_t xs = static_cast<size_t>(M) * K * 2, ys = static_cast<size_t>(M) * N * 2;
+  if (xb < yb + ys && yb < xb + xs) return fail(LL_ERR_INVALID_ARG);
+  if (!is_device_ptr(x) || !is_device_ptr(y) || !is_device_ptr(Q) || !is_device_ptr(scale) ||
+      (bias && !is_device_ptr(bias)) || (r > 0 && (!is_device_ptr(A) || !is_device_ptr(B))))
+    return fail(LL_ERR_INVALID_ARG);
+  const int rc = forward_noalloc(x, A, B, Q, scale, scale_mode, bias, y, M, N, K, r, static_cast<cudaStream_t>(stream));
+  return rc == LL_OK ? LL_OK : fail(rc);
+}

@@ -85,3 +85,18 @@ def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_noalloc_argument_checks_need_no_gpu():
+    """ll_forward_noalloc rejects bad shapes and modes before any CUDA call."""
+    import rank_fp8_residual_b200 as ll
+    f = ll._lib.ll_forward_noalloc
+    P = None
+    assert f(P, P, P, P, P, 1, P, P, 0, 64, 64, 8, P) == ll.LL_OK          # M == 0 is a no-op
+    assert f(P, P, P, P, P, 1, P, P, 4, 60, 64, 8, P) == ll.LL_ERR_INVALID_ARG   # N % 8
+    assert f(P, P, P, P, P, 1, P, P, 4, 64, 40, 8, P) == ll.LL_ERR_INVALID_ARG   # K % 16
+    assert f(P, P, P, P, P, 1, P, P, 4, 64, 64, 513, P) == ll.LL_ERR_INVALID_ARG  # r > 512
+    assert f(P, P, P, P, P, 5, P, P, 4, 64, 64, 8, P) == ll.LL_ERR_INVALID_ARG   # scale mode
+    assert f(P, P, P, P, P, 1, P, P, 4, 64, 64, 12, P) == ll.LL_ERR_UNSUPPORTED  # r % 8
+    assert f(P, P, P, P, P, 1, P, P, 4, 64, 64, 8, P) == ll.LL_ERR_INVALID_ARG   # null pointers
+    assert ll.ll_last_error() == ll.LL_ERR_INVALID_ARG
