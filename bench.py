@@ -73,19 +73,29 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+# Sources each kernel is compiled from: a recorded ncu capture stays valid
+# while these files are unchanged.
+KERNEL_SOURCES = {
+    "ll_tc_kernel": ["ll_tc.cuh", "ll_kernels.cuh", "ptx.cuh"],
+    "ll_tc2_kernel": ["ll_tc2.cuh", "ll_kernels.cuh", "ptx.cuh"],
+    "ll_main_kernel": ["ll_kernels.cuh", "ptx.cuh"],
+    "ll_lrdown_kernel": ["ll_kernels.cuh", "ptx.cuh"],
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rank_fp8_residual_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(n.encode() + f.read())
+    names = KERNEL_SOURCES.get(kernel) or sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh")))
+    for n in names:
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu capture, or None when the
-    kernel sources changed since the capture."""
+    kernel's sources changed since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -93,7 +103,7 @@ def recorded_traffic(kernel, workload):
     except (OSError, ValueError):
         return None
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
