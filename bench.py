@@ -80,6 +80,7 @@ KERNEL_SOURCES = {
     "ll_tc2_kernel": ["ll_tc2.cuh", "ll_kernels.cuh", "ptx.cuh"],
     "ll_main_kernel": ["ll_kernels.cuh", "ptx.cuh"],
     "ll_lrdown_kernel": ["ll_kernels.cuh", "ptx.cuh"],
+    "ll_stream_kernel": ["ll_stream.cuh", "ll_kernels.cuh", "ptx.cuh"],
 }
 
 
@@ -237,7 +238,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="auto", choices=["auto", "tc", "tc_pair", "small"],
+    ap.add_argument("--variant", default="auto", choices=["auto", "tc", "tc_pair", "small", "stream"],
                     help="kernel variant (auto picks by token count)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -270,7 +271,7 @@ def main():
                       inp.bias.to(dev) if inp.bias is not None else None)
     h = layer.handle
     ll.ll_set_variant(h, {"auto": ll.LL_VARIANT_AUTO, "tc": ll.LL_VARIANT_TC, "tc_pair": ll.LL_VARIANT_TC_PAIR,
-                          "small": ll.LL_VARIANT_SMALL}[args.variant])
+                          "small": ll.LL_VARIANT_SMALL, "stream": ll.LL_VARIANT_STREAM}[args.variant])
     ll.ll_reserve(h, w.M)
     x = inp.x.to(dev)
     y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)

@@ -64,14 +64,22 @@ enum {
   LL_ERR_SCRATCH_LIMIT = 8   /* request too large for ll_forward_noalloc's scratch */
 };
 
-/* Kernel variants for ll_set_variant.  AUTO: TC for M > 128, SMALL
- * otherwise.  TC: one-CTA fused kernel, 128 features x 256 tokens per
- * tile, low-rank factor folded as A / scale (bf16 pair).  TC_PAIR: the
- * same on CTA pairs (256 features per MMA); slower than TC on every
- * measured shape, kept selectable for comparison.  SMALL: one-CTA kernel,
- * 128 x 128 tiles, separate residual and low-rank accumulators.  Every
+/* Kernel variants for ll_set_variant.  AUTO: STREAM for M <= 64, SMALL
+ * for 64 < M <= 128, TC above.  TC: one-CTA fused kernel, 128 features x
+ * 256 tokens per tile, low-rank factor folded as A / scale (bf16 pair).
+ * TC_PAIR: the same on CTA pairs (256 features per MMA); slower than TC on
+ * every measured shape, kept selectable for comparison.  SMALL: one-CTA
+ * kernel, 128 x 128 tiles, separate residual and low-rank accumulators.
+ * STREAM (M <= 64 only; larger M runs SMALL): one CTA per 128 features
+ * streaming Q in 32 KB boxes, all tokens in one MMA, exact A.  Every
  * variant meets the same accuracy bound. */
-enum { LL_VARIANT_AUTO = 0, LL_VARIANT_TC = 1, LL_VARIANT_SMALL = 2, LL_VARIANT_TC_PAIR = 3 };
+enum {
+  LL_VARIANT_AUTO = 0,
+  LL_VARIANT_TC = 1,
+  LL_VARIANT_SMALL = 2,
+  LL_VARIANT_TC_PAIR = 3,
+  LL_VARIANT_STREAM = 4
+};
 
 /* Create a layer with N output features, K input features and rank r on
  * the current CUDA device.  Requires N >= 1 and N % 8 == 0, K >= 16 and
@@ -168,9 +176,9 @@ const char *ll_kernel_name(ll_handle h, int i);
  * factors into library-owned memory) or ll_forward (it grows a workspace
  * on demand).  This call takes no handle: the caller passes every input
  * and the output, and the intermediate t = x B^T (bf16 hi + lo), its
- * split-K partial sums, a device status word and, for a per-tensor scale,
- * the scale broadcast to N rows live in one static device array of
- * LL_NOALLOC_SCRATCH_BYTES.  Every GPU on which the library's device code
+ * split-K partial sums and arrival counters, a device status word and,
+ * for a per-tensor scale, the scale broadcast to N rows live in one static
+ * device array of LL_NOALLOC_SCRATCH_BYTES.  Every GPU on which the library's device code
  * is loaded holds that array until the process exits.
  *
  * y is the forward of ll_forward with the SMALL variant (residual and
@@ -198,7 +206,8 @@ const char *ll_kernel_name(ll_handle h, int i);
  *
  * Shared scratch: every call on a device uses the same array, and the
  * array keeps the last call's contents.  Each call clears the status word
- * and fully rewrites t before reading it.  Calls whose kernels overlap on
+ * and fully rewrites t before reading it; the split-K counters start at
+ * zero when the library loads and every call leaves them at zero.  Calls whose kernels overlap on
  * the GPU (issued on two streams without ordering, or from two host
  * threads) race on the array and give wrong results: order them on one
  * stream or with events.

@@ -34,6 +34,7 @@ LL_VARIANT_AUTO = 0
 LL_VARIANT_TC = 1
 LL_VARIANT_SMALL = 2
 LL_VARIANT_TC_PAIR = 3
+LL_VARIANT_STREAM = 4
 
 # Every symbol the header declares, with (restype, argtypes).
 _P = ctypes.c_void_p

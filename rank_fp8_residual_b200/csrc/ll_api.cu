@@ -17,6 +17,7 @@
 #include "ll_kernels.cuh"
 #include "ll_tc.cuh"
 #include "ll_tc2.cuh"
+#include "ll_stream.cuh"
 
 namespace {
 
@@ -115,6 +116,7 @@ struct ll_layer {
   int* status = nullptr;      // device status word
   int* flags = nullptr;       // [2] set-time scan flags
   int* sched = nullptr;       // [2] tile scheduler of the fused kernel
+  int* lr_cnt = nullptr;      // [kLrMaxTiles] split-K arrival counters of the down-projection
   // workspace for t
   int ws_M = 0;
   uint16_t* t_hi = nullptr;
@@ -133,6 +135,7 @@ struct ll_layer {
   void* c_yptr = nullptr;
   int c_M = -1;
   CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256, c_thik, c_tlok, c_x3;
+  CUtensorMap c_xs, c_this, c_tlos;  // streaming kernel: x and t boxes of Mt rows
   CUtensorMap tm_q3;  // 3-D view of the (row-cleared) residual, 4 K chunks per box
   int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
   int variant = LL_VARIANT_AUTO;
@@ -163,6 +166,7 @@ void free_layer_mem(ll_layer* h) {
   cudaFree(h->status);
   cudaFree(h->flags);
   cudaFree(h->sched);
+  cudaFree(h->lr_cnt);
   cudaFree(h->t_hi);
   cudaFree(h->t_lo);
   cudaFree(h->part);
@@ -186,6 +190,9 @@ int set_smem_attrs_once() {
       rc = 1;
     if (cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::lr_smem_bytes(256)) != cudaSuccess)
+      rc = 1;
+    if (cudaFuncSetAttribute(llk::ll_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::st_smem_max()) != cudaSuccess)
       rc = 1;
   });
   return rc;
@@ -227,14 +234,21 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
   return LL_OK;
 }
 
-enum Path { PATH_SMALL, PATH_TC1, PATH_TC2 };
+enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM };
+
+constexpr int kStreamMaxM = 64;
 
 Path choose_path(const ll_layer* h, int M) {
   if (h->variant == LL_VARIANT_TC) return PATH_TC1;
   if (h->variant == LL_VARIANT_TC_PAIR) return PATH_TC2;
   if (h->variant == LL_VARIANT_SMALL) return PATH_SMALL;
+  if (h->variant == LL_VARIANT_STREAM) return M <= kStreamMaxM ? PATH_STREAM : PATH_SMALL;
+  if (M <= kStreamMaxM) return PATH_STREAM;
   return M > 128 ? PATH_TC1 : PATH_SMALL;
 }
+
+// CTAs of the streaming kernel: one per 128-feature tile, at most one per SM.
+int stream_ctas(const ll_layer* h) { return std::min((h->N + 127) / 128, h->num_sms); }
 
 // The CTA-pair kernel computes t with the warp-level kernel beside it.
 bool warp_lowrank(const ll_layer* h, int M) {
@@ -269,9 +283,14 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   const int ctas = p.m_tiles * p.r_chunks;
   // With the single-CTA fused kernel the down-projection runs beside it on
   // a quarter of the SMs; the other kernels wait for it, so it takes all.
-  const int budget = path == PATH_TC1 ? std::max(1, h->num_sms / 4) : h->num_sms;
+  // The streaming kernel leaves the SMs beyond its tiles to the
+  // down-projection, which runs beside it.
+  int budget = h->num_sms;
+  if (path == PATH_TC1) budget = std::max(1, h->num_sms / 4);
+  if (path == PATH_STREAM) budget = std::max(1, h->num_sms - stream_ctas(h));
   int ks = std::max(1, budget / ctas);
-  ks = std::min(ks, nK);
+  ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);
+  if (ctas > llk::kLrMaxTiles) ks = 1;
   p.kb_per_split = (nK + ks - 1) / ks;
   p.ksplit = (nK + p.kb_per_split - 1) / p.kb_per_split;
   return p;
@@ -292,6 +311,17 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   ok &= make_map(&h->c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (h->K % 64 == 0) ok &= make_map3(&h->c_x3, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, 128, 2,
                                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (M <= kStreamMaxM) {
+    const uint32_t Mt = static_cast<uint32_t>((M + 15) / 16 * 16);
+    if (h->K % 64 == 0)
+      ok &= make_map3(&h->c_xs, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, Mt, 4, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+      ok &= make_map(&h->c_xs, x, kBF16, M, h->K, 2ull * h->K, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (h->r_pad > 0) {
+      ok &= make_map(&h->c_this, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&h->c_tlos, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+  }
   if (h->r_pad > 0) {
     const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     ok &= make_map(&h->c_thi128, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -372,6 +402,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     lpp.t_hi = h->t_hi;
     lpp.t_lo = h->t_lo;
     lpp.part = h->part;
+    lpp.cnt = h->lr_cnt;
     lpp.M = M;
     lpp.K = h->K;
     lpp.r_pad = h->r_pad;
@@ -384,13 +415,6 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     ll_lrdown_kernel<<<grid, kLrThreads, lr_smem_bytes(lp.rc), st>>>(lpp);
     h->names[launches++] = "ll_lrdown_kernel";
     if (prof) cudaEventRecord(h->ev[launches], st);
-    if (lp.ksplit > 1) {
-      const size_t total4 = static_cast<size_t>(M) * h->r_pad / 4;
-      int blocks = static_cast<int>(std::min<size_t>((total4 + 255) / 256, static_cast<size_t>(h->num_sms) * 4));
-      ll_lrsplit_kernel<<<blocks, 256, 0, st>>>(h->part, h->t_hi, h->t_lo, M, h->r_pad, lp.ksplit);
-      h->names[launches++] = "ll_lrsplit_kernel";
-      if (prof) cudaEventRecord(h->ev[launches], st);
-    }
     if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
   }
 
@@ -405,7 +429,33 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   cfg.attrs = attr;
   cfg.numAttrs = overlap ? 1 : 0;
   cudaError_t err;
-  if (path == PATH_TC2) {
+  if (path == PATH_STREAM) {
+    StreamParams sp;
+    const bool dims3 = h->K % 64 == 0;
+    sp.tm_x = h->c_xs;
+    sp.tm_q = dims3 ? h->tm_q3 : h->tm_q;
+    sp.tm_a = h->tm_a;
+    sp.tm_thi = h->c_this;
+    sp.tm_tlo = h->c_tlos;
+    sp.scale = h->scale;
+    sp.bias = h->has_bias ? h->bias : nullptr;
+    sp.y = static_cast<uint16_t*>(y);
+    sp.M = M;
+    sp.N = h->N;
+    sp.K = h->K;
+    sp.r_pad = h->r_pad;
+    sp.Mt = (M + 15) / 16 * 16;
+    sp.n_ftiles = (h->N + 127) / 128;
+    sp.dims3 = dims3 ? 1 : 0;
+    sp.lr_from_primary = overlap ? 1 : 0;
+    sp.withhold = h->withhold;
+    sp.watch = watch;
+    cfg.gridDim = dim3(stream_ctas(h));
+    cfg.blockDim = dim3(kStThreads);
+    cfg.dynamicSmemBytes = st_smem_bytes(sp.Mt);
+    err = cudaLaunchKernelEx(&cfg, ll_stream_kernel, sp);
+    h->names[launches] = "ll_stream_kernel";
+  } else if (path == PATH_TC2) {
     Tc2Params tp;
     tp.dims3 = h->K % 64 == 0 ? 1 : 0;
     tp.tm_x = tp.dims3 ? h->c_x3 : h->c_x128;
@@ -575,6 +625,7 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
   ok &= cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
   ok &= cudaMalloc(&h->flags, 2 * sizeof(int)) == cudaSuccess;
   ok &= cudaMalloc(&h->sched, 2 * sizeof(int)) == cudaSuccess;
+  ok &= cudaMalloc(&h->lr_cnt, llk::kLrMaxTiles * sizeof(int)) == cudaSuccess;
   if (h->r_pad > 0) {
     ok &= cudaMalloc(&h->A, sizeof(uint16_t) * nrp) == cudaSuccess;
     ok &= cudaMalloc(&h->Ahi, sizeof(uint16_t) * nrp) == cudaSuccess;
@@ -591,6 +642,7 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
   h->Qf = h->Q;
   cudaMemset(h->status, 0, sizeof(int));
   cudaMemset(h->sched, 0, 2 * sizeof(int));
+  cudaMemset(h->lr_cnt, 0, llk::kLrMaxTiles * sizeof(int));
   using namespace llk;
   ok &= make_map(&h->tm_q, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
   h->tm_qf = h->tm_q;
@@ -783,7 +835,7 @@ int ll_reserve(ll_handle h, int max_M) {
 int ll_set_variant(ll_handle h, int variant) {
   g_last_error = LL_OK;
   if (!h || (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC && variant != LL_VARIANT_SMALL &&
-             variant != LL_VARIANT_TC_PAIR))
+             variant != LL_VARIANT_TC_PAIR && variant != LL_VARIANT_STREAM))
     return fail(LL_ERR_INVALID_ARG);
   h->variant = variant;
   return LL_OK;
@@ -799,9 +851,11 @@ int ll_status(ll_handle h) {
     return fail(LL_ERR_CUDA);
   }
   if (v != 0) {
-    // A kernel gave up part-way: clear the status and the tile scheduler.
+    // A kernel gave up part-way: clear the status, the tile scheduler and
+    // the split-K counters.
     cudaMemset(h->status, 0, sizeof(int));
     cudaMemset(h->sched, 0, 2 * sizeof(int));
+    cudaMemset(h->lr_cnt, 0, llk::kLrMaxTiles * sizeof(int));
     cudaDeviceSynchronize();
     return LL_ERR_DEVICE_TIMEOUT;
   }
@@ -932,8 +986,10 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   NoAllocDevice* d = noalloc_setup(dev, &rc);
   if (!d) return rc;
 
-  // Scratch layout: status word | broadcast scale (per-tensor only) |
-  // t_hi [M, r_pad] | t_lo [M, r_pad] | split-K partials (what is left).
+  // Scratch layout: status word (bytes 0-3) and split-K arrival counters
+  // (bytes 64-255, kept at zero between calls) | broadcast scale
+  // (per-tensor only) | t_hi [M, r_pad] | t_lo [M, r_pad] | split-K
+  // partials (what is left).
   const int r_pad = (r + 31) / 32 * 32;
   const size_t t_bytes = static_cast<size_t>(M) * r_pad * sizeof(uint16_t);
   size_t off = 256;
@@ -946,6 +1002,8 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
 
   unsigned char* base = d->scratch;
   int* status = reinterpret_cast<int*>(base);
+  int* lr_cnt = reinterpret_cast<int*>(base + 64);
+  constexpr int kCounters = (256 - 64) / static_cast<int>(sizeof(int));
   const float* scale_n = scale;
   if (scale_mode == LL_SCALE_PER_TENSOR) scale_n = reinterpret_cast<float*>(base + scale_off);
   uint16_t* t_hi = reinterpret_cast<uint16_t*>(base + thi_off);
@@ -962,6 +1020,10 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   view.num_sms = d->num_sms;
   view.variant = LL_VARIANT_SMALL;
   LrPlan lp = plan_lowrank(&view, M);
+  if (lp.ksplit > 1 && lp.m_tiles * lp.r_chunks > kCounters) {
+    lp.kb_per_split = (K + kBK - 1) / kBK;
+    lp.ksplit = 1;
+  }
   if (r_pad > 0 && lp.ksplit > 1) {
     const size_t per_split = static_cast<size_t>(M) * r_pad * sizeof(float);
     const size_t fit = (LL_NOALLOC_SCRATCH_BYTES - part_off) / per_split;
@@ -1007,6 +1069,7 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
     lpp.t_hi = t_hi;
     lpp.t_lo = t_lo;
     lpp.part = part;
+    lpp.cnt = lr_cnt;
     lpp.M = M;
     lpp.K = K;
     lpp.r_pad = r_pad;
@@ -1017,12 +1080,6 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
     lpp.watch = watch;
     dim3 grid(lp.m_tiles, lp.r_chunks, lp.ksplit);
     ll_lrdown_kernel<<<grid, kLrThreads, lr_smem_bytes(lp.rc), st>>>(lpp);
-    if (lp.ksplit > 1) {
-      const size_t total4 = static_cast<size_t>(M) * r_pad / 4;
-      const int blocks =
-          static_cast<int>(std::min<size_t>((total4 + 255) / 256, static_cast<size_t>(d->num_sms) * 4));
-      ll_lrsplit_kernel<<<blocks, 256, 0, st>>>(part, t_hi, t_lo, M, r_pad, lp.ksplit);
-    }
   }
   if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
 

@@ -9,13 +9,12 @@
 // factor shapes).
 //
 // Kernel chain for one forward (all on the caller's stream):
-//   1. ll_lrdown_kernel   t = x B^T with tcgen05, fp32 accumulate in TMEM.
-//                         With one K split it writes t as a bf16 pair
-//                         (t_hi = bf16(t), t_lo = bf16(t - t_hi)); with
-//                         several K splits it writes fp32 partial sums.
-//   2. ll_lrsplit_kernel  (only with K splits) sums the partials in a fixed
-//                         order and writes the bf16 pair.
-//   3. ll_main_kernel     persistent fused GEMM.  Tile = 128 output
+//   1. ll_lrdown_kernel   t = x B^T with tcgen05, fp32 accumulate in TMEM,
+//                         written as a bf16 pair (t_hi = bf16(t),
+//                         t_lo = bf16(t - t_hi)).  With several K splits
+//                         each CTA writes an fp32 partial sum and the last
+//                         CTA of a tile adds them in split order.
+//   2. ll_main_kernel     persistent fused GEMM.  Tile = 128 output
 //                         features x up to 128 tokens.  Q (e4m3fn) is the
 //                         MMA A operand: converter warps widen it exactly to
 //                         bf16 and write it into tensor memory; x is the MMA
@@ -25,7 +24,7 @@
 //                         y = scale[n]*acc_Q + acc_LR + bias[n] in fp32,
 //                         rounds once to bf16 and writes with TMA stores.
 //                         It is launched with programmatic dependent launch
-//                         and waits for kernels 1/2 only before its first
+//                         and waits for kernel 1 only before its first
 //                         read of t, so its x*Q^T main loop overlaps them.
 #pragma once
 #include <cstdint>
@@ -72,6 +71,7 @@ struct LrDownParams {
   uint16_t* t_hi;    // [M, r_pad] bf16 bits
   uint16_t* t_lo;    // [M, r_pad]
   float* part;       // [ksplit, M, r_pad] fp32 (ksplit > 1)
+  int* cnt;          // [gridDim.x * gridDim.y] arrival counters, zero between calls (ksplit > 1)
   int M, K, r_pad;
   int rc;            // box height of B = column block of t per CTA (<= 256)
   int tmem_cols;     // power of two >= rc
@@ -82,6 +82,8 @@ struct LrDownParams {
 
 constexpr int kLrStages = 4;
 constexpr int kLrThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr int kLrMaxSplit = 8;   // K splits per tile (the last CTA of a tile sums them)
+constexpr int kLrMaxTiles = 1024;  // tiles with split K (arrival counters)
 
 __host__ __device__ constexpr int lr_stage_bytes(int rc) { return 128 * kBK * 2 + rc * kBK * 2; }
 __host__ constexpr int lr_smem_bytes(int rc) { return kLrStages * lr_stage_bytes(rc) + 1024 + 256; }
@@ -217,41 +219,67 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
       }
     }
   }
+  if (p.ksplit > 1) __threadfence();  // partials visible before this CTA counts itself in
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, ncols);
   }
-}
+  if (p.ksplit == 1) return;
 
-// Kernel 2: sum the K-split partials of t in split order and write the
-// bf16 pair.  One thread per 4 consecutive elements.
-__global__ void ll_lrsplit_kernel(const float* __restrict__ part, uint16_t* __restrict__ t_hi,
-                                  uint16_t* __restrict__ t_lo, int M, int r_pad, int ksplit) {
-  pdl_launch_dependents();
-  const size_t total4 = static_cast<size_t>(M) * r_pad / 4;
-  const size_t plane = static_cast<size_t>(M) * r_pad;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total4;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    float4 acc = reinterpret_cast<const float4*>(part)[i];
-    for (int z = 1; z < ksplit; ++z) {
-      const float4 v = reinterpret_cast<const float4*>(part + z * plane)[i];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+  // Split K: the last CTA of this tile to arrive sums the partials in
+  // split order and writes the bf16 pair, then re-arms the counter.  Every
+  // CTA counts itself in, also after a timeout, so the counter is back at
+  // zero when the grid ends.
+  __shared__ int s_last;
+  int* cnt = p.cnt + blockIdx.y * gridDim.x + blockIdx.x;
+  if (threadIdx.x == 0) s_last = atomicAdd(cnt, 1) == p.ksplit - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int rows = min(128, p.M - m0);
+  const int q4 = wcols / 4;
+  const int total = rows * q4;
+  const size_t plane = static_cast<size_t>(p.M) * p.r_pad;
+  // Each thread sums kLrRedPer float4 columns at once, with every partial
+  // load issued before the first add (the sums are latency-bound).
+  constexpr int kLrRedPer = 4;
+  for (int i0 = threadIdx.x; i0 < total; i0 += kLrRedPer * blockDim.x) {
+    float4 v[kLrRedPer][kLrMaxSplit];
+    size_t off[kLrRedPer];
+#pragma unroll
+    for (int u = 0; u < kLrRedPer; ++u) {
+      const int i = i0 + u * blockDim.x;
+      off[u] = i < total ? static_cast<size_t>(m0 + i / q4) * p.r_pad + j0 + 4 * (i % q4) : 0;
+#pragma unroll
+      for (int z = 0; z < kLrMaxSplit; ++z)
+        if (i < total && z < p.ksplit) v[u][z] = __ldcg(reinterpret_cast<const float4*>(p.part + z * plane + off[u]));
     }
-    const uint16_t h0 = to_bf16_bits(acc.x), h1 = to_bf16_bits(acc.y);
-    const uint16_t h2 = to_bf16_bits(acc.z), h3 = to_bf16_bits(acc.w);
-    uint2 hv, lv;
-    hv.x = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-    hv.y = static_cast<uint32_t>(h2) | (static_cast<uint32_t>(h3) << 16);
-    lv.x = pack_bf16x2(acc.x - bf16_bits_to_float(h0), acc.y - bf16_bits_to_float(h1));
-    lv.y = pack_bf16x2(acc.z - bf16_bits_to_float(h2), acc.w - bf16_bits_to_float(h3));
-    reinterpret_cast<uint2*>(t_hi)[i] = hv;
-    reinterpret_cast<uint2*>(t_lo)[i] = lv;
+#pragma unroll
+    for (int u = 0; u < kLrRedPer; ++u) {
+      if (i0 + u * static_cast<int>(blockDim.x) >= total) break;
+      float4 acc = v[u][0];
+#pragma unroll
+      for (int z = 1; z < kLrMaxSplit; ++z)
+        if (z < p.ksplit) {
+          acc.x += v[u][z].x;
+          acc.y += v[u][z].y;
+          acc.z += v[u][z].z;
+          acc.w += v[u][z].w;
+        }
+      const uint16_t h0 = to_bf16_bits(acc.x), h1 = to_bf16_bits(acc.y);
+      const uint16_t h2 = to_bf16_bits(acc.z), h3 = to_bf16_bits(acc.w);
+      uint2 hv, lv;
+      hv.x = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+      hv.y = static_cast<uint32_t>(h2) | (static_cast<uint32_t>(h3) << 16);
+      lv.x = pack_bf16x2(acc.x - bf16_bits_to_float(h0), acc.y - bf16_bits_to_float(h1));
+      lv.y = pack_bf16x2(acc.z - bf16_bits_to_float(h2), acc.w - bf16_bits_to_float(h3));
+      *reinterpret_cast<uint2*>(p.t_hi + off[u]) = hv;
+      *reinterpret_cast<uint2*>(p.t_lo + off[u]) = lv;
+    }
   }
+  if (threadIdx.x == 0) *cnt = 0;
 }
 
 // =====================================================================

@@ -180,6 +180,20 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]
       : "r"(taddr)
       : "memory");
 }
+// Two 16-column loads (from two TMEM addresses) with one wait.
+__device__ __forceinline__ void tmem_ld16x2_wait(uint32_t ta, uint32_t (&r)[16], uint32_t tb, uint32_t (&s)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : LLK_R8(0), LLK_R8(8), "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
+        "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]), "=r"(s[12]), "=r"(s[13]),
+        "=r"(s[14]), "=r"(s[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
 // Two 32-column loads (from two TMEM addresses) with one wait.
 __device__ __forceinline__ void tmem_ld32x2_wait(uint32_t ta, uint32_t (&r)[32], uint32_t tb,
                                                  uint32_t (&s)[32]) {

@@ -19,8 +19,10 @@ pytestmark = pytest.mark.gpu
 
 
 VARIANTS = [ll.LL_VARIANT_TC, ll.LL_VARIANT_SMALL, ll.LL_VARIANT_TC_PAIR]
+# The streaming variant serves M <= 64 only (larger M runs the SMALL kernel).
+SMALL_M_VARIANTS = VARIANTS + [ll.LL_VARIANT_STREAM]
 VNAME = {ll.LL_VARIANT_TC: "tc", ll.LL_VARIANT_SMALL: "small", ll.LL_VARIANT_AUTO: "auto",
-         ll.LL_VARIANT_TC_PAIR: "tc-pair"}
+         ll.LL_VARIANT_TC_PAIR: "tc-pair", ll.LL_VARIANT_STREAM: "stream"}
 
 
 def _full(inp, what, variant=ll.LL_VARIANT_AUTO):
@@ -44,6 +46,27 @@ def test_widening_is_exact_for_every_code(variant):
     y = run(inp, variant).to(torch.float64)
     expect = codes.view(torch.float8_e4m3fn).to(torch.float64).t()  # [M=K, N]
     assert torch.equal(y, expect)
+
+
+@pytest.mark.parametrize("K", [256, 272])
+def test_widening_is_exact_for_every_code_streaming(K):
+    """The same check for the streaming kernel, which takes at most 64
+    tokens: four calls of 64 one-hot tokens cover all K positions (K = 272
+    exercises the 2-D loads of a K that is not a multiple of 64)."""
+    N = 256
+    n = torch.arange(N).view(N, 1)
+    k = torch.arange(K).view(1, K)
+    codes = ((n + k) % 256).to(torch.uint8)
+    codes[(codes == 0x7F) | (codes == 0xFF)] = 0
+    expect_all = codes.view(torch.float8_e4m3fn).to(torch.float64).t()  # [K, N]
+    for k0 in range(0, K, 64):
+        M = min(64, K - k0)
+        x = torch.zeros(M, K, dtype=torch.bfloat16)
+        x[torch.arange(M), k0 + torch.arange(M)] = 1.0
+        inp = LayerInputs(M, K, N, 0, SCALE_PER_TENSOR, x, None, None, codes,
+                          torch.ones(1, dtype=torch.float32), None)
+        y = run(inp, ll.LL_VARIANT_STREAM).to(torch.float64)
+        assert torch.equal(y, expect_all[k0:k0 + M])
 
 
 def test_tiny_config():
@@ -98,10 +121,32 @@ def test_scale_far_outside_fold_range_is_rejected():
         ll.ll_destroy(h)
 
 
-@pytest.mark.parametrize("variant", VARIANTS)
-@pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 31, 64])
+@pytest.mark.parametrize("variant", SMALL_M_VARIANTS)
+@pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 31, 33, 48, 63, 64])
 def test_small_token_counts(M, variant):
     _full(make_inputs(M, 512, 1024, 96, seed=10 + M), f"M={M}", variant)
+
+
+@pytest.mark.parametrize("M,K,N,r", [(5, 272, 392, 40), (40, 1024, 136, 64), (64, 384, 1000, 200),
+                                     (17, 4096, 2056, 512), (64, 2048, 20480, 32)])
+def test_streaming_ragged(M, K, N, r):
+    """Ragged feature tails, K not a multiple of 64, every rank chunking,
+    and more feature tiles than SMs (persistent CTAs)."""
+    inp = make_inputs(M, K, N, r, scale_range=(1e-3, 3e-3), seed=M + N)
+    inp.scale[::11] = 0.0
+    _full(inp, f"stream {M}x{K}x{N} r{r}", ll.LL_VARIANT_STREAM)
+
+
+@pytest.mark.parametrize("variant", [ll.LL_VARIANT_STREAM])
+@pytest.mark.parametrize("case", ["r0", "q0", "per_tensor_no_bias"])
+def test_streaming_special_cases(case, variant):
+    if case == "r0":
+        inp = make_inputs(50, 256, 256, 0, seed=51)
+    elif case == "q0":
+        inp = make_inputs(50, 256, 256, 32, seed=52, q_zero=True)
+    else:
+        inp = make_inputs(45, 320, 264, 24, scale_mode=SCALE_PER_TENSOR, bias=False, seed=53)
+    _full(inp, f"stream {case}", variant)
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
@@ -114,6 +159,11 @@ def test_token_tile_edges(M, variant):
 @pytest.mark.parametrize("r", [1, 31, 32, 33, 63, 64, 65, 96, 128, 160, 256, 320, 512])
 def test_rank_edges(r, variant):
     _full(make_inputs(300, 256, 256, r, seed=30 + r), f"r={r}", variant)
+
+
+@pytest.mark.parametrize("r", [1, 33, 64, 65, 160, 512])
+def test_rank_edges_streaming(r):
+    _full(make_inputs(37, 256, 256, r, seed=60 + r), f"stream r={r}", ll.LL_VARIANT_STREAM)
 
 
 def test_attention_projection_full():
