@@ -137,6 +137,9 @@ struct ll_layer {
   CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256, c_thik, c_tlok, c_x3;
   CUtensorMap c_xs, c_this, c_tlos;  // streaming kernel: x and t boxes of Mt rows
   CUtensorMap tm_q3;  // 3-D view of the (row-cleared) residual, 4 K chunks per box
+  CUtensorMap tm_q3b2;  // the same view, 2 K chunks per box (fused single-CTA kernel)
+  CUtensorMap c_xbt, c_thibt, c_tlobt;  // fused single-CTA kernel: x and t boxes of bt rows
+  int c_bt = 0;
   int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
   int variant = LL_VARIANT_AUTO;
   int withhold = 0;
@@ -250,6 +253,27 @@ Path choose_path(const ll_layer* h, int M) {
 // CTAs of the streaming kernel: one per 128-feature tile, at most one per SM.
 int stream_ctas(const ll_layer* h) { return std::min((h->N + 127) / 128, h->num_sms); }
 
+// Tokens per tile of the single-CTA fused kernel: the multiple of 32 up to
+// 256 that finishes the tiles in the least time per SM, modelled as waves
+// of num_sms tiles times (tile width + a fixed per-tile cost worth about 80
+// token columns: the epilogue and the pipeline fill); ties go to the wider
+// tile.
+int tc_tile_tokens(const ll_layer* h, int M) {
+  constexpr int kTileCost = 80;
+  const int n_ftiles = (h->N + 127) / 128;
+  int best = 256;
+  long long best_cost = -1;
+  for (int bt = 256; bt >= 128; bt -= 32) {
+    const long long tiles = static_cast<long long>(n_ftiles) * ((M + bt - 1) / bt);
+    const long long cost = (tiles + h->num_sms - 1) / h->num_sms * (bt + kTileCost);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bt;
+    }
+  }
+  return best;
+}
+
 // The CTA-pair kernel computes t with the warp-level kernel beside it.
 bool warp_lowrank(const ll_layer* h, int M) {
   return choose_path(h, M) == PATH_TC2 && h->r_pad > 0 && h->r_pad <= 128;
@@ -283,10 +307,13 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   const int ctas = p.m_tiles * p.r_chunks;
   // With the single-CTA fused kernel the down-projection runs beside it on
   // a quarter of the SMs; the other kernels wait for it, so it takes all.
-  // The streaming kernel leaves the SMs beyond its tiles to the
-  // down-projection, which runs beside it.
+  // The down-projection runs beside the fused kernels: on half of the SMs
+  // next to the large-M kernel (whose CTAs take tiles from a shared
+  // counter, so those that start late take fewer), and on the SMs the
+  // streaming kernel's tiles leave free.  The other kernels wait for it, so
+  // it takes all SMs.
   int budget = h->num_sms;
-  if (path == PATH_TC1) budget = std::max(1, h->num_sms / 4);
+  if (path == PATH_TC1) budget = std::max(1, h->num_sms / 2);
   if (path == PATH_STREAM) budget = std::max(1, h->num_sms - stream_ctas(h));
   int ks = std::max(1, budget / ctas);
   ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);
@@ -311,6 +338,16 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   ok &= make_map(&h->c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (h->K % 64 == 0) ok &= make_map3(&h->c_x3, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, 128, 2,
                                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (M > 128) {
+    const int bt = tc_tile_tokens(h, M);
+    h->c_bt = bt;
+    ok &= make_map(&h->c_xbt, x, kBF16, M, h->K, 2ull * h->K, kBK, bt, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (h->r_pad > 0) {
+      const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+      ok &= make_map(&h->c_thibt, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
+      ok &= make_map(&h->c_tlobt, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
+    }
+  }
   if (M <= kStreamMaxM) {
     const uint32_t Mt = static_cast<uint32_t>((M + 15) / 16 * 16);
     if (h->K % 64 == 0)
@@ -490,12 +527,15 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     h->names[launches] = "ll_tc2_kernel";
   } else if (path == PATH_TC1) {
     TcParams tp;
-    tp.tm_x = h->c_x256;
-    tp.tm_q = h->tm_qf;
+    const bool large = M > 128;  // the per-call maps of bt rows exist for M > 128
+    tp.bt = large ? h->c_bt : 256;
+    tp.tm_x = large ? h->c_xbt : h->c_x256;
+    tp.q3 = h->K % 64 == 0 ? 1 : 0;
+    tp.tm_q = tp.q3 ? h->tm_q3b2 : h->tm_qf;
     tp.tm_ahi = h->tm_ahi;
     tp.tm_alo = h->tm_alo;
-    tp.tm_thi = h->c_thi256;
-    tp.tm_tlo = h->c_tlo256;
+    tp.tm_thi = large ? h->c_thibt : h->c_thi256;
+    tp.tm_tlo = large ? h->c_tlobt : h->c_tlo256;
     tp.tm_y = h->c_y;
     tp.scale = h->scale_eff;
     tp.bias = h->has_bias ? h->bias : nullptr;
@@ -506,7 +546,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     tp.r_pad = h->r_pad;
     tp.klr = h->klr;
     tp.n_ftiles = (h->N + 127) / 128;
-    tp.n_ttiles = (M + kTcBT - 1) / kTcBT;
+    tp.n_ttiles = (M + tp.bt - 1) / tp.bt;
     tp.lr_from_primary = overlap ? 1 : 0;
     tp.withhold = h->withhold;
     tp.watch = watch;
@@ -646,9 +686,12 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
   using namespace llk;
   ok &= make_map(&h->tm_q, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
   h->tm_qf = h->tm_q;
-  if (K % 64 == 0)
+  if (K % 64 == 0) {
     ok &= make_map3(&h->tm_q3, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
                     CU_TENSOR_MAP_SWIZZLE_64B);
+    ok &= make_map3(&h->tm_q3b2, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 2,
+                    CU_TENSOR_MAP_SWIZZLE_64B);
+  }
   if (h->r_pad > 0) {
     const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     ok &= make_map(&h->tm_a, h->A, kBF16, N, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -721,9 +764,12 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
       ok &= cudaMalloc(&h->Qf, nq) == cudaSuccess;
       ok &= make_map(&h->tm_qf, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, llk::kBK, 128,
                      CU_TENSOR_MAP_SWIZZLE_64B);
-      if (K % 64 == 0)
+      if (K % 64 == 0) {
         ok &= make_map3(&h->tm_q3, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
                         CU_TENSOR_MAP_SWIZZLE_64B);
+        ok &= make_map3(&h->tm_q3b2, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 2,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+      }
     }
     if (ok) {
       llk::ll_zero_rows_kernel<<<h->num_sms * 8, 256>>>(h->Q, h->scale, h->Qf, N, K);
@@ -733,9 +779,12 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
     cudaFree(h->Qf);
     h->Qf = h->Q;
     h->tm_qf = h->tm_q;
-    if (K % 64 == 0)
+    if (K % 64 == 0) {
       ok &= make_map3(&h->tm_q3, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
                       CU_TENSOR_MAP_SWIZZLE_64B);
+      ok &= make_map3(&h->tm_q3b2, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 2,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
+    }
   }
   if (rp > 0) {
     ok &= cudaMemset(h->A, 0, sizeof(uint16_t) * N * static_cast<size_t>(rp)) == cudaSuccess;

@@ -80,21 +80,28 @@ struct LrDownParams {
   Watch watch;
 };
 
-constexpr int kLrStages = 4;
+// Ring depth: as many stages as fit in 192 KB (4 to 8): t's reads of x come
+// from HBM, so the more bytes in flight the closer to its bandwidth.
+constexpr int kLrMaxStages = 8;
+constexpr int kLrRingBytes = 192 * 1024;
 constexpr int kLrThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 constexpr int kLrMaxSplit = 8;   // K splits per tile (the last CTA of a tile sums them)
 constexpr int kLrMaxTiles = 1024;  // tiles with split K (arrival counters)
 
 __host__ __device__ constexpr int lr_stage_bytes(int rc) { return 128 * kBK * 2 + rc * kBK * 2; }
-__host__ constexpr int lr_smem_bytes(int rc) { return kLrStages * lr_stage_bytes(rc) + 1024 + 256; }
+__host__ __device__ constexpr int lr_stages(int rc) {
+  return kLrRingBytes / lr_stage_bytes(rc) < kLrMaxStages ? kLrRingBytes / lr_stage_bytes(rc) : kLrMaxStages;
+}
+__host__ constexpr int lr_smem_bytes(int rc) { return lr_stages(rc) * lr_stage_bytes(rc) + 1024 + 256; }
 
 __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_constant__ LrDownParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int stage_bytes = lr_stage_bytes(p.rc);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kLrStages * stage_bytes);
-  uint64_t* empty = full + kLrStages;
-  uint64_t* acc_full = empty + kLrStages;
+  const int n_stages = lr_stages(p.rc);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + n_stages * stage_bytes);
+  uint64_t* empty = full + n_stages;
+  uint64_t* acc_full = empty + n_stages;
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
@@ -110,7 +117,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     pdl_launch_dependents();
-    for (int s = 0; s < kLrStages; ++s) {
+    for (int s = 0; s < n_stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -142,12 +149,12 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
         tma_load_2d(st, &p.tm_x, &full[s], kb * kBK, m0);
         tma_load_2d(st + 128 * kBK * 2, &p.tm_b, &full[s], kb * kBK, j0);
         ++issued;
-        if (++s == kLrStages) { s = 0; ph ^= 1; }
+        if (++s == n_stages) { s = 0; ph ^= 1; }
       }
       if (!ok) {
         // Let every load already issued land before the CTA can exit.
-        for (int i = max(0, issued - kLrStages); i < issued; ++i)
-          mbar_wait_drain(&full[i % kLrStages], (i / kLrStages) & 1, p.watch);
+        for (int i = max(0, issued - n_stages); i < issued; ++i)
+          mbar_wait_drain(&full[i % n_stages], (i / n_stages) & 1, p.watch);
       }
     }
   } else if (warp == 1) {
@@ -168,7 +175,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
           first = false;
         }
         tc_commit(&empty[s]);
-        if (++s == kLrStages) { s = 0; ph ^= 1; }
+        if (++s == n_stages) { s = 0; ph ^= 1; }
       }
       tc_commit(acc_full);
       // No MMA may still run when TMEM is released below.

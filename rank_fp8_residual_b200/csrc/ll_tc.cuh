@@ -17,16 +17,21 @@
 // low-rank term.  Rows with s[n] == 0 use s = 1 and an all-zero residual row
 // (exact, since 0 * (x Q^T) = 0).
 //
-// Tile: 128 output features (MMA M, TMEM lanes) x up to 256 tokens (MMA N,
-// TMEM columns).  Q is the MMA A operand: eight converter warps widen the
-// e4m3fn codes exactly to bf16 and store them into TMEM stages; x is the B
-// operand, staged by TMA.  Persistent CTAs take tiles from a device-wide
-// counter in a grouped raster order (8 token tiles per group) so that the
-// tiles in flight share their x and Q slabs in L2.
+// Tile: 128 output features (MMA M, TMEM lanes) x bt tokens (MMA N, TMEM
+// columns; bt <= 256, a multiple of 16 chosen per call so that the tiles
+// fill the SMs in as few equal waves as possible).  Q is the MMA A operand:
+// eight converter warps widen the e4m3fn codes exactly to bf16 and store
+// them into TMEM stages of two K steps (64 columns); x is the B operand,
+// staged by TMA.  Persistent CTAs take tiles from a device-wide counter in a
+// grouped raster order (8 token tiles per group) so that the tiles in flight
+// share their x and Q slabs in L2.  Every tile, the first included, comes
+// from that counter.
 //
-// Warp roles (14 warps): 0 TMA producer + tile scheduler, 1 MMA issuer
-// (also allocates TMEM), 2-9 converters (lane quadrant w%4, K half
-// (w-2)/4), 10-13 epilogue (lane quadrant w%4).
+// Warp roles (15 warps): 0 TMA producer of Q + tile scheduler, 1 MMA issuer
+// (also allocates TMEM), 2-9 converters (lane quadrant w%4, K step parity
+// (w-2)/4 within a stage), 10-13 epilogue (lane quadrant w%4), 14 TMA
+// producer of x and of the low-rank A' / t chunks.  The two producers are
+// separate so that each ring runs ahead on its own.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -37,49 +42,55 @@
 namespace llk {
 
 struct TcParams {
-  CUtensorMap tm_x;    // bf16 [M, K]       box {64, 256},  128B swizzle
-  CUtensorMap tm_q;    // u8   [N, K]       box {64, 128},   64B swizzle
+  CUtensorMap tm_x;    // bf16 [M, K]       box {64, bt},   128B swizzle
+  CUtensorMap tm_q;    // u8   [N, K]       3-D {64, N, K/64} box {64, 128, 2}, or 2-D box {64, 128}; 64B swizzle
   CUtensorMap tm_ahi;  // bf16 [N, r_pad]   box {klr, 128}, 128B (klr 64) / 64B (klr 32) swizzle
   CUtensorMap tm_alo;  // bf16 [N, r_pad]
-  CUtensorMap tm_thi;  // bf16 [M, r_pad]   box {klr, 256}
+  CUtensorMap tm_thi;  // bf16 [M, r_pad]   box {klr, bt}
   CUtensorMap tm_tlo;  // bf16 [M, r_pad]
   CUtensorMap tm_y;    // bf16 [M, N]       box {32, 32},    no swizzle
   const float* scale;    // effective per-row scale [N]
   const uint16_t* bias;  // [N] bf16 bits, or nullptr
   int* sched;            // [2]: tile counter, finished-CTA counter (0 between launches)
   int M, N, K, r_pad, klr;
+  int bt;                // tokens per tile (multiple of 16, <= 256)
   int n_ftiles, n_ttiles;
+  int q3;                // 1: one 3-D Q load per stage; 0: two 2-D loads
   int lr_from_primary;
   int withhold;
   Watch watch;
 };
 
-constexpr int kTcThreads = 448;
-constexpr int kTcBT = 256;                  // tokens per tile
-constexpr int kTcSX = 4;                    // 32 KB slots: x chunks, A'/t chunks
-constexpr int kTcSQ = 6;                    // 8 KB slots: Q chunks
-constexpr int kTcNA = 8;                    // widened-Q stages in TMEM (32 columns each)
-constexpr int kTcXSlot = kTcBT * kBK * 2;   // 32768
-constexpr int kTcQSlot = 128 * kBK;         // 8192
-constexpr int kTcEpi = 4 * 2 * 32 * 32 * 2; // 4 warps x 2 buffers x (32 tokens x 32 features) bf16
-constexpr int kTcGroup = 8;                 // token tiles per raster group
 constexpr int kTcConvWarps = 8;
 constexpr int kTcEpiWarps = 4;
+constexpr int kTcXWarp = 2 + kTcConvWarps + kTcEpiWarps;  // x / low-rank producer
+constexpr int kTcThreads = 32 * (kTcXWarp + 1);
+constexpr int kTcMaxBT = 256;               // tokens per tile, at most
+constexpr int kTcSX = 4;                    // 32 KB slots: x chunks, A'/t chunks
+constexpr int kTcSQ = 4;                    // 16 KB slots: Q, two K steps each
+constexpr int kTcNA = 4;                    // widened-Q stages in TMEM (two K steps, 64 columns each)
+constexpr int kTcXSlot = kTcMaxBT * kBK * 2;  // 32768
+constexpr int kTcQChunk = 128 * kBK;        // 8192: 128 rows x 64 codes
+constexpr int kTcQSlot = 2 * kTcQChunk;
+constexpr int kTcEpi = 4 * 2 * 32 * 32 * 2; // 4 warps x 2 buffers x (32 tokens x 32 features) bf16
+constexpr int kTcGroup = 8;                 // token tiles per raster group
 constexpr int kTcTileRing = 2;
 constexpr int kTcColA = 256;                // TMEM column of the first widened-Q stage
+// Consumers of a scheduled tile: MMA, converters, epilogue, x producer.
+constexpr int kTcTileUsers = 1 + kTcConvWarps + kTcEpiWarps + 1;
 
 __host__ __device__ constexpr int tc_smem_bytes() {
   return kTcSX * kTcXSlot + kTcSQ * kTcQSlot + kTcEpi + 1024 + 512;
 }
 
-__device__ __forceinline__ void tc_tile_coords(int T, int n_ftiles, int n_ttiles, int& f0, int& t0) {
+__device__ __forceinline__ void tc_tile_coords(int T, int n_ftiles, int n_ttiles, int bt, int& f0, int& t0) {
   const int per_group = kTcGroup * n_ftiles;
   const int g = T / per_group;
   const int first_tt = g * kTcGroup;
   const int gsize = min(kTcGroup, n_ttiles - first_tt);
   const int idx = T - g * per_group;
   f0 = (idx / gsize) * 128;
-  t0 = (first_tt + idx % gsize) * kTcBT;
+  t0 = (first_tt + idx % gsize) * bt;
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_constant__ TcParams p) {
@@ -105,8 +116,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = p.n_ftiles * p.n_ttiles;
   const int nK = (p.K + kBK - 1) / kBK;
+  const int nS = (nK + 1) / 2;  // stages of two K steps (a step past K loads as zeros)
   const int nR = p.r_pad / p.klr;
   const int klr = p.klr;
+  const int bt = p.bt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcSX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
@@ -116,7 +129,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     mbar_init(acc_empty, kTcEpiWarps);
     for (int s = 0; s < kTcTileRing; ++s) {
       mbar_init(&tile_full[s], 1);
-      mbar_init(&tile_empty[s], 1 + kTcConvWarps + kTcEpiWarps);
+      mbar_init(&tile_empty[s], kTcTileUsers);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -140,37 +153,77 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
   const uint32_t tbase = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------- TMA + tile scheduler
+    // --------------------------------------------- TMA: Q + tile scheduler
     if (lane == 0) {
-      int xi = 0, qi = 0, ti = 0;
-      uint32_t xph = 0, qph = 0, tph = 0;
-      long long nx = 0, nq = 0;
-      bool ok = true, waited_primary = false;
-      int T = blockIdx.x;
-      const uint32_t a_bytes = 128u * klr * 2u;
-      const uint32_t t_bytes = static_cast<uint32_t>(kTcBT) * klr * 2u;
+      int qi = 0, ti = 0;
+      uint32_t qph = 0, tph = 0;
+      long long nq = 0;
+      bool ok = true;
       for (;;) {
         if (!mbar_wait(&tile_empty[ti], tph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+        // Every tile, the first included, comes from the shared counter, so
+        // a CTA that starts late (its SM still busy with the kernel before)
+        // simply takes fewer tiles.
+        const int T = atomicAdd(&p.sched[0], 1);
         const bool live = T < n_tiles;
         *reinterpret_cast<volatile int*>(&tile_slot[ti]) = live ? T : -1;
         mbar_arrive(&tile_full[ti]);
         if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
         if (!live) break;
         if (p.withhold) { ok = false; break; }  // debug: no loads, the consumers time out
-        const int next = static_cast<int>(gridDim.x) + atomicAdd(&p.sched[0], 1);
         int f0, t0;
-        tc_tile_coords(T, p.n_ftiles, p.n_ttiles, f0, t0);
-        for (int kb = 0; kb < nK && ok; ++kb) {
+        tc_tile_coords(T, p.n_ftiles, p.n_ttiles, bt, f0, t0);
+        for (int s = 0; s < nS; ++s) {
+          if (!mbar_wait(&q_empty[qi], qph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+          uint8_t* dst = sq + qi * kTcQSlot;
+          mbar_arrive_expect_tx(&q_full[qi], kTcQSlot);
+          if (p.q3) {
+            tma_load_3d(dst, &p.tm_q, &q_full[qi], 0, f0, 2 * s);
+          } else {
+            tma_load_2d(dst, &p.tm_q, &q_full[qi], 2 * s * kBK, f0);
+            tma_load_2d(dst + kTcQChunk, &p.tm_q, &q_full[qi], (2 * s + 1) * kBK, f0);
+          }
+          ++nq;
+          if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      if (!ok) {
+        for (long long i = (nq > kTcSQ ? nq - kTcSQ : 0); i < nq; ++i)
+          mbar_wait_drain(&q_full[i % kTcSQ], static_cast<uint32_t>((i / kTcSQ) & 1), p.watch);
+      }
+      // The last CTA to finish resets the scheduler for the next launch.
+      __threadfence();
+      if (atomicAdd(&p.sched[1], 1) == static_cast<int>(gridDim.x) - 1) {
+        atomicExch(&p.sched[0], 0);
+        atomicExch(&p.sched[1], 0);
+      }
+    }
+  } else if (warp == kTcXWarp) {
+    // --------------------------------- TMA: x, then A' and t chunks (L2)
+    if (lane == 0) {
+      int xi = 0, ti = 0;
+      uint32_t xph = 0, tph = 0;
+      long long nx = 0;
+      bool ok = true, waited_primary = false;
+      const uint32_t x_bytes = static_cast<uint32_t>(bt) * kBK * 2u;
+      const uint32_t a_bytes = 128u * klr * 2u;
+      const uint32_t t_bytes = static_cast<uint32_t>(bt) * klr * 2u;
+      for (;;) {
+        if (!mbar_wait(&tile_full[ti], tph, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+        const int T = *reinterpret_cast<volatile int*>(&tile_slot[ti]);
+        mbar_arrive(&tile_empty[ti]);
+        if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
+        if (T < 0) break;
+        if (p.withhold) { ok = false; break; }
+        int f0, t0;
+        tc_tile_coords(T, p.n_ftiles, p.n_ttiles, bt, f0, t0);
+        for (int kb = 0; kb < 2 * nS && ok; ++kb) {
           if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&x_full[xi], kTcXSlot);
+          mbar_arrive_expect_tx(&x_full[xi], x_bytes);
           tma_load_2d(sx + xi * kTcXSlot, &p.tm_x, &x_full[xi], kb * kBK, t0);
           ++nx;
           if (++xi == kTcSX) { xi = 0; xph ^= 1; }
-          if (!mbar_wait(&q_empty[qi], qph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&q_full[qi], kTcQSlot);
-          tma_load_2d(sq + qi * kTcQSlot, &p.tm_q, &q_full[qi], kb * kBK, f0);
-          ++nq;
-          if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
         }
         if (ok && nR > 0 && !waited_primary && p.lr_from_primary) {
           pdl_wait_primary();
@@ -196,19 +249,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
           if (++xi == kTcSX) { xi = 0; xph ^= 1; }
         }
         if (!ok) break;
-        T = next;
       }
       if (!ok) {
         for (long long i = (nx > kTcSX ? nx - kTcSX : 0); i < nx; ++i)
           mbar_wait_drain(&x_full[i % kTcSX], static_cast<uint32_t>((i / kTcSX) & 1), p.watch);
-        for (long long i = (nq > kTcSQ ? nq - kTcSQ : 0); i < nq; ++i)
-          mbar_wait_drain(&q_full[i % kTcSQ], static_cast<uint32_t>((i / kTcSQ) & 1), p.watch);
-      }
-      // The last CTA to finish resets the scheduler for the next launch.
-      __threadfence();
-      if (atomicAdd(&p.sched[1], 1) == static_cast<int>(gridDim.x) - 1) {
-        atomicExch(&p.sched[0], 0);
-        atomicExch(&p.sched[1], 0);
       }
     }
   } else if (warp == 1) {
@@ -225,23 +269,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
         if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
         if (T < 0) break;
         int f0, t0;
-        tc_tile_coords(T, p.n_ftiles, p.n_ttiles, f0, t0);
-        const int valid = min(kTcBT, p.M - t0);
+        tc_tile_coords(T, p.n_ftiles, p.n_ttiles, bt, f0, t0);
+        const int valid = min(bt, p.M - t0);
         const uint32_t idesc = idesc_bf16(128, (valid + 15) & ~15);
         if (!mbar_wait(acc_empty, accph ^ 1, p.watch, kErrTimeoutMma)) break;
         tc_fence_after();
-        for (int kb = 0; kb < nK; ++kb) {
+        for (int s = 0; s < nS && ok; ++s) {
           if (!mbar_wait(&a_full[ai], aph, p.watch, kErrTimeoutMma)) { ok = false; break; }
-          if (!mbar_wait(&x_full[xi], xph, p.watch, kErrTimeoutMma)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sx + xi * kTcXSlot));
-          const uint32_t at = tbase + kTcColA + ai * 32;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_ts(tbase, at + kk * 8, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-          tc_commit(&x_empty[xi]);
+          for (int sub = 0; sub < 2; ++sub) {
+            if (!mbar_wait(&x_full[xi], xph, p.watch, kErrTimeoutMma)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sx + xi * kTcXSlot));
+            const uint32_t at = tbase + kTcColA + ai * 64 + sub * 32;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              mma_ts(tbase, at + kk * 8, bd + 2 * kk, idesc, (s | sub | kk) != 0 ? 1u : 0u);
+            tc_commit(&x_empty[xi]);
+            if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          }
+          if (!ok) break;
           tc_commit(&a_empty[ai]);
-          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
           if (++ai == kTcNA) { ai = 0; aph ^= 1; }
         }
         for (int jb = 0; jb < nR && ok; ++jb) {
@@ -280,11 +328,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     }
   } else if (warp < 2 + kTcConvWarps) {
     // ----------------------------------------- e4m3 -> bf16 into TMEM stages
+    // Warp (q, par) widens K step 2s + par of every stage s for the rows of
+    // lane quadrant q: one full 64-code row chunk per lane.
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;           // which 32 of the 64 K columns
+    const int par = (warp - 2) >> 2;
     const int row = 32 * q + lane;              // feature row within the tile
     const int sw = (row >> 1) & 3;              // 64-byte swizzle phase of the row
-    const uint32_t tl = tbase + ((32u * q) << 16) + kTcColA + 16 * half;
+    const uint32_t tl = tbase + ((32u * q) << 16) + kTcColA + 32 * par;
     int qi = 0, ai = 0, ti = 0;
     uint32_t qph = 0, aph = 0, tph = 0;
     bool ok = true;
@@ -295,36 +345,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
       if (lane == 0) mbar_arrive(&tile_empty[ti]);
       if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
       if (T < 0) break;
-      // Software pipeline: the codes of step kb+1 are read from shared
-      // memory before step kb is stored into TMEM.
-      uint4 v0, v1;
+      // Software pipeline: the codes of stage s+1 are read from shared
+      // memory before stage s is stored into TMEM.
+      uint4 v[4];
+      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qi], qph, p.watch, kErrTimeoutConvert))) break;
       {
-        if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qi], qph, p.watch, kErrTimeoutConvert))) break;
-        const uint8_t* rb = sq + qi * kTcQSlot + row * 64;
-        v0 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half) ^ sw));
-        v1 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half + 1) ^ sw));
+        const uint8_t* rb = sq + qi * kTcQSlot + par * kTcQChunk + row * 64;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(rb + 16 * (j ^ sw));
         __syncwarp();
         if (lane == 0) mbar_arrive(&q_empty[qi]);
         if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
       }
-      for (int kb = 0; kb < nK; ++kb) {
-        uint32_t w[16];
-        e4m3x4_to_bf16x4(v0.x, w[0], w[1]);
-        e4m3x4_to_bf16x4(v0.y, w[2], w[3]);
-        e4m3x4_to_bf16x4(v0.z, w[4], w[5]);
-        e4m3x4_to_bf16x4(v0.w, w[6], w[7]);
-        e4m3x4_to_bf16x4(v1.x, w[8], w[9]);
-        e4m3x4_to_bf16x4(v1.y, w[10], w[11]);
-        e4m3x4_to_bf16x4(v1.z, w[12], w[13]);
-        e4m3x4_to_bf16x4(v1.w, w[14], w[15]);
-        if (kb + 1 < nK) {
+      for (int s = 0; s < nS; ++s) {
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          e4m3x4_to_bf16x4(v[j].x, w[8 * j + 0], w[8 * j + 1]);
+          e4m3x4_to_bf16x4(v[j].y, w[8 * j + 2], w[8 * j + 3]);
+          e4m3x4_to_bf16x4(v[j].z, w[8 * j + 4], w[8 * j + 5]);
+          e4m3x4_to_bf16x4(v[j].w, w[8 * j + 6], w[8 * j + 7]);
+        }
+        if (s + 1 < nS) {
           if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qi], qph, p.watch, kErrTimeoutConvert))) {
             ok = false;
             break;
           }
-          const uint8_t* rb = sq + qi * kTcQSlot + row * 64;
-          v0 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half) ^ sw));
-          v1 = *reinterpret_cast<const uint4*>(rb + 16 * ((2 * half + 1) ^ sw));
+          const uint8_t* rb = sq + qi * kTcQSlot + par * kTcQChunk + row * 64;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(rb + 16 * (j ^ sw));
           __syncwarp();
           if (lane == 0) mbar_arrive(&q_empty[qi]);
           if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
@@ -334,8 +383,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
           break;
         }
         tc_fence_after();
-        tmem_st16(tl + ai * 32, w);
-        tmem_st_wait();
+        tmem_st32_wait(tl + ai * 64, w);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[ai]);
@@ -343,7 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
       }
       if (!ok) break;
     }
-  } else {
+  } else if (warp < kTcXWarp) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int frow = 32 * q + lane;
@@ -359,8 +407,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
       if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
       if (T < 0) break;
       int f0, t0;
-      tc_tile_coords(T, p.n_ftiles, p.n_ttiles, f0, t0);
-      const int valid = min(kTcBT, p.M - t0);
+      tc_tile_coords(T, p.n_ftiles, p.n_ttiles, bt, f0, t0);
+      const int valid = min(bt, p.M - t0);
       const int f = f0 + frow;
       const float s = f < p.N ? p.scale[f] : 0.f;
       const float b = (p.bias != nullptr && f < p.N) ? bf16_bits_to_float(p.bias[f]) : 0.f;
