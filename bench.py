@@ -30,7 +30,6 @@ this build) on the same workload, metric and unit.
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import math
@@ -248,22 +247,20 @@ def main():
         return run_reference(args, w)
 
     import torch
-    import torch.distributed as dist
     import rank_fp8_residual_b200 as ll
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from rank_fp8_residual_b200 import replicas
+    rank, world, local_rank = replicas.rank_env()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        replicas.init("nccl", device=dev)
 
     # Factors are shared (seed 0); each rank draws its own tokens.
     inp = w.inputs(seed=0)
     if rank != 0:
         from synth_inputs import make_x
-        inp.x = make_x(w.M, w.K, seed=1000 + rank)
+        inp.x = make_x(w.M, w.K, seed=replicas.token_seed(rank))
     layer = ll.LiteLinearLayer(w.N, w.K, w.r, w.scale_mode)
     layer.set_weights(inp.A.to(dev) if inp.A is not None else None,
                       inp.B.to(dev) if inp.B is not None else None,
@@ -279,16 +276,10 @@ def main():
     stream = torch.cuda.Stream(device=dev)
     flops, bytes_, main_flops, main_bytes = work_of(w)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = replicas.barrier
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, device=dev)
 
     # --------------------------------------------------- device-timed steps
     with torch.cuda.stream(stream):
@@ -316,7 +307,7 @@ def main():
     st = ll.ll_status(h)
     if st != ll.LL_OK:
         raise SystemExit(f"device status after timing: {ll.status_string(st)}")
-    value = world * args.steps * flops / (total_ms * 1e-3) / 1e12
+    value = replicas.aggregate_rate(flops, args.steps, total_ms * 1e-3, world) / 1e12
 
     # ------------------------------------------- end to end (host buffers)
     xh = inp.x.contiguous().pin_memory()
@@ -393,8 +384,8 @@ def main():
         line["cpu_baseline"] = cpu_baseline(w)
     layer.close()
     if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+        replicas.barrier()
+        replicas.finalize()
     if rank == 0:
         print(json.dumps(line))
     return 0
