@@ -27,10 +27,14 @@
 // share their x and Q slabs in L2.  Every tile, the first included, comes
 // from that counter.
 //
-// Warp roles (15 warps): 0 TMA producer of Q + tile scheduler, 1 MMA issuer
-// (also allocates TMEM), 2-9 converters (lane quadrant w%4, K step parity
-// (w-2)/4 within a stage), 10-13 epilogue (lane quadrant w%4), 14 TMA
-// producer of x and of the low-rank A' / t chunks.  The two producers are
+// Warp roles (27 warps): 0 TMA producer of Q + tile scheduler, 1 MMA issuer
+// (also allocates TMEM), 2-17 converters in two teams of eight that take
+// alternate stages (lane quadrant w%4, K step parity within a stage), so
+// four converter warps share each SM sub-partition and hide one another's
+// shared-memory, barrier and TMEM-store latency, 18-25 epilogue (lane
+// quadrant w%4, two warps per quadrant on alternate 32-token blocks, so the
+// accumulator is free for the next tile sooner), 26 TMA producer of x and
+// of the low-rank A' / t chunks.  The two producers are
 // separate so that each ring runs ahead on its own.
 #pragma once
 #include <cstdint>
@@ -61,8 +65,8 @@ struct TcParams {
   Watch watch;
 };
 
-constexpr int kTcConvWarps = 8;
-constexpr int kTcEpiWarps = 4;
+constexpr int kTcConvWarps = 16;  // two teams of 8; team t widens the stages of parity t
+constexpr int kTcEpiWarps = 8;   // two per lane quadrant, alternate 32-token blocks
 constexpr int kTcXWarp = 2 + kTcConvWarps + kTcEpiWarps;  // x / low-rank producer
 constexpr int kTcThreads = 32 * (kTcXWarp + 1);
 constexpr int kTcMaxBT = 256;               // tokens per tile, at most
@@ -72,7 +76,7 @@ constexpr int kTcNA = 4;                    // widened-Q stages in TMEM (two K s
 constexpr int kTcXSlot = kTcMaxBT * kBK * 2;  // 32768
 constexpr int kTcQChunk = 128 * kBK;        // 8192: 128 rows x 64 codes
 constexpr int kTcQSlot = 2 * kTcQChunk;
-constexpr int kTcEpi = 4 * 2 * 32 * 32 * 2; // 4 warps x 2 buffers x (32 tokens x 32 features) bf16
+constexpr int kTcEpi = kTcEpiWarps * 2 * 32 * 32 * 2;
 constexpr int kTcGroup = 8;                 // token tiles per raster group
 constexpr int kTcTileRing = 2;
 constexpr int kTcColA = 256;                // TMEM column of the first widened-Q stage
@@ -123,8 +127,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcSX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
-    for (int s = 0; s < kTcSQ; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], kTcConvWarps); }
-    for (int s = 0; s < kTcNA; ++s) { mbar_init(&a_full[s], kTcConvWarps); mbar_init(&a_empty[s], 1); }
+    // A Q slot and a TMEM stage each hold one stage, which one team reads / writes.
+    for (int s = 0; s < kTcSQ; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], kTcConvWarps / 2); }
+    for (int s = 0; s < kTcNA; ++s) { mbar_init(&a_full[s], kTcConvWarps / 2); mbar_init(&a_empty[s], 1); }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kTcEpiWarps);
     for (int s = 0; s < kTcTileRing; ++s) {
@@ -328,15 +333,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     }
   } else if (warp < 2 + kTcConvWarps) {
     // ----------------------------------------- e4m3 -> bf16 into TMEM stages
-    // Warp (q, par) widens K step 2s + par of every stage s for the rows of
-    // lane quadrant q: one full 64-code row chunk per lane.
+    // Stages are numbered across this CTA's tiles (g); team t takes the
+    // stages g = t (mod 2).  Within a team, warp (q, par) widens K step
+    // 2s + par of the stage for the rows of lane quadrant q: one full
+    // 64-code row chunk per lane.  Stage g uses Q slot and TMEM stage
+    // g mod 4, in phase (g / 4) mod 2.
+    static_assert(kTcSQ == kTcNA, "Q slots and TMEM stages advance together");
+    const int cw = warp - 2;
+    const int team = cw >> 3;
     const int q = warp & 3;
-    const int par = (warp - 2) >> 2;
+    const int par = (cw >> 2) & 1;
     const int row = 32 * q + lane;              // feature row within the tile
     const int sw = (row >> 1) & 3;              // 64-byte swizzle phase of the row
     const uint32_t tl = tbase + ((32u * q) << 16) + kTcColA + 32 * par;
-    int qi = 0, ai = 0, ti = 0;
-    uint32_t qph = 0, aph = 0, tph = 0;
+    int ti = 0;
+    uint32_t tph = 0;
+    long long gs = 0;  // stages of this CTA before the current tile
     bool ok = true;
     for (;;) {
       if (!__all_sync(0xffffffffu, mbar_wait(&tile_full[ti], tph, p.watch, kErrTimeoutConvert))) break;
@@ -345,19 +357,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
       if (lane == 0) mbar_arrive(&tile_empty[ti]);
       if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
       if (T < 0) break;
-      // Software pipeline: the codes of stage s+1 are read from shared
-      // memory before stage s is stored into TMEM.
-      uint4 v[4];
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qi], qph, p.watch, kErrTimeoutConvert))) break;
-      {
-        const uint8_t* rb = sq + qi * kTcQSlot + par * kTcQChunk + row * 64;
+      for (long long g = gs + ((team - gs) & 1); g < gs + nS; g += 2) {
+        const int slot = static_cast<int>(g % kTcSQ);
+        const uint32_t ph = static_cast<uint32_t>((g / kTcSQ) & 1);
+        if (!__all_sync(0xffffffffu, mbar_wait(&q_full[slot], ph, p.watch, kErrTimeoutConvert))) { ok = false; break; }
+        uint4 v[4];
+        const uint8_t* rb = sq + slot * kTcQSlot + par * kTcQChunk + row * 64;
 #pragma unroll
         for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(rb + 16 * (j ^ sw));
         __syncwarp();
-        if (lane == 0) mbar_arrive(&q_empty[qi]);
-        if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
-      }
-      for (int s = 0; s < nS; ++s) {
+        if (lane == 0) mbar_arrive(&q_empty[slot]);
         uint32_t w[32];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -366,30 +375,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
           e4m3x4_to_bf16x4(v[j].z, w[8 * j + 4], w[8 * j + 5]);
           e4m3x4_to_bf16x4(v[j].w, w[8 * j + 6], w[8 * j + 7]);
         }
-        if (s + 1 < nS) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qi], qph, p.watch, kErrTimeoutConvert))) {
-            ok = false;
-            break;
-          }
-          const uint8_t* rb = sq + qi * kTcQSlot + par * kTcQChunk + row * 64;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(rb + 16 * (j ^ sw));
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&q_empty[qi]);
-          if (++qi == kTcSQ) { qi = 0; qph ^= 1; }
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[ai], aph ^ 1, p.watch, kErrTimeoutConvert))) {
-          ok = false;
-          break;
-        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[slot], ph ^ 1, p.watch, kErrTimeoutConvert))) { ok = false; break; }
         tc_fence_after();
-        tmem_st32_wait(tl + ai * 64, w);
+        tmem_st32_wait(tl + slot * 64, w);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[ai]);
-        if (++ai == kTcNA) { ai = 0; aph ^= 1; }
+        if (lane == 0) mbar_arrive(&a_full[slot]);
       }
       if (!ok) break;
+      gs += nS;
     }
   } else if (warp < kTcXWarp) {
     // ------------------------------------------------------------ epilogue
@@ -397,6 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     const int frow = 32 * q + lane;
     const uint32_t tl = tbase + ((32u * q) << 16);
     uint16_t* stage = reinterpret_cast<uint16_t*>(se + (warp - 2 - kTcConvWarps) * (2 * 32 * 32 * 2));
+    const int eh = (warp - 2 - kTcConvWarps) >> 2;  // which 32-token blocks: parity eh
     int eb = 0, ti = 0;
     uint32_t accph = 0, tph = 0;
     for (;;) {
@@ -415,7 +410,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
       if (!__all_sync(0xffffffffu, mbar_wait(acc_full, accph, p.watch, kErrTimeoutEpilogue))) break;
       tc_fence_after();
       const bool store_rows = f0 + 32 * q < p.N;
-      for (int c = 0; c < valid; c += 32) {
+      for (int c = 32 * eh; c < valid; c += 64) {
         uint32_t v[32];
         tmem_ld32_wait(tl + c, v);
         if (lane == 0) tma_store_wait_read<1>();
