@@ -229,6 +229,76 @@ def run_reference(args, w):
     return 0
 
 
+def run_page_suite(args):
+    """The FFN shapes of the LiteLinear README's LTX-Video benchmark table
+    (its "Performance Benchmark on shapes captured from LTX-Video" section):
+    every (projection, M) row timed on its own, and the count-weighted total
+    of the rows, which is the table's TOTAL row (in ms)."""
+    import torch
+    import rank_fp8_residual_b200 as ll
+    from synth_inputs import PAGE_MICROBENCH, page_workload
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    steps = max(1, min(args.steps, 30))
+    rows, total_ms, total_flops_calls = [], 0.0, 0.0
+    layers = {}
+    for cfg, m, count in PAGE_MICROBENCH:
+        w = WORKLOADS[page_workload(cfg, m, args.rank)]
+        key = (w.K, w.N)
+        if key not in layers:  # one layer per projection: the factors do not depend on M
+            B, A, Q, scale, bias = w.weights(seed=0)
+            layer = ll.LiteLinearLayer(w.N, w.K, w.r, w.scale_mode)
+            layer.set_weights(A.to(dev), B.to(dev), Q.to(dev), scale.to(dev), bias.to(dev))
+            layers[key] = layer
+        h = layers[key].handle
+        ll.ll_reserve(h, w.M)
+        # Activations drawn on the device (the largest row block is 1.4 GB).
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 + m)
+        x = torch.randn(w.M, w.K, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+        ev = []
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup + steps):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                ll.ll_forward(h, x, y, w.M, stream)
+                b.record(stream)
+                if i >= args.warmup:
+                    ev.append((a, b))
+        torch.cuda.synchronize()
+        st = ll.ll_status(h)
+        if st != ll.LL_OK:
+            raise SystemExit(f"device status: {ll.status_string(st)}")
+        us = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+        med = us[len(us) // 2]
+        flops = work_of(w)[0]
+        rows.append({"cfg": cfg, "M": m, "K": w.K, "N": w.N, "count": count, "us": round(med, 2),
+                     "tflops": round(flops / (med * 1e-6) / 1e12, 1)})
+        total_ms += count * med * 1e-3
+        total_flops_calls += count * flops
+        del x, y
+    for layer in layers.values():
+        layer.close()
+    line = {
+        "metric": "LTX-Video FFN shapes, count-weighted total time", "value": total_ms, "unit": "ms",
+        "higher_is_better": False, "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"page_microbench_r{args.rank}", "rank": args.rank,
+                   "reading": "w1 = 4096 -> 16384, w2 = 16384 -> 4096 (K, N not on the page)",
+                   "l2": "flushed between calls (256 MiB write, outside the events)", "rows": rows},
+        "tflops_weighted": total_flops_calls / (total_ms * 1e-3) / 1e12,
+        "vs_baseline": None,
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -239,9 +309,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", default="auto", choices=["auto", "tc", "tc_pair", "small", "stream"],
                     help="kernel variant (auto picks by token count)")
+    ap.add_argument("--suite", default=None, choices=["page"],
+                    help="page: the README's LTX-Video FFN shapes, count-weighted total (one GPU)")
+    ap.add_argument("--rank", type=int, default=64, choices=[32, 64], help="rank of the --suite shapes")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.suite == "page":
+        return run_page_suite(args)
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

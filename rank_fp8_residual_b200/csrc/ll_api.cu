@@ -307,13 +307,13 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   const int ctas = p.m_tiles * p.r_chunks;
   // With the single-CTA fused kernel the down-projection runs beside it on
   // a quarter of the SMs; the other kernels wait for it, so it takes all.
-  // The down-projection runs beside the fused kernels: on half of the SMs
-  // next to the large-M kernel (whose CTAs take tiles from a shared
+  // The down-projection runs beside the fused kernels: on three quarters of
+  // the SMs next to the large-M kernel (whose CTAs take tiles from a shared
   // counter, so those that start late take fewer), and on the SMs the
   // streaming kernel's tiles leave free.  The other kernels wait for it, so
   // it takes all SMs.
   int budget = h->num_sms;
-  if (path == PATH_TC1) budget = std::max(1, h->num_sms / 2);
+  if (path == PATH_TC1) budget = std::max(1, h->num_sms * 3 / 4);
   if (path == PATH_STREAM) budget = std::max(1, h->num_sms - stream_ctas(h));
   int ks = std::max(1, budget / ctas);
   ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);

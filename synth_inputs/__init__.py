@@ -149,7 +149,34 @@ def _build_workloads():
             for r in (32, 64, 512):
                 name = f"sweep_m{m}_k{k}_n{n}_r{r}"
                 w[name] = Workload(name, m, k, n, r)
+    # The FFN shapes captured from LTX-Video that the LiteLinear README's
+    # kernel benchmark lists ("Performance Benchmark on shapes captured from
+    # LTX-Video"): w1 = up-projection, w2 = down-projection, M = flattened
+    # activation rows.  The page states neither K / N nor the rank; the
+    # shapes here take the README's own usage example (in_features 4096,
+    # out_features 16384) for the up-projection and its transpose for the
+    # down-projection, at ranks 32 and 64.
+    for cfg, m, _count in PAGE_MICROBENCH:
+        k, n = (4096, 16384) if cfg == "w1" else (16384, 4096)
+        for r in (32, 64):
+            name = f"page_{cfg}_m{m}_k{k}_n{n}_r{r}"
+            w[name] = Workload(name, m, k, n, r)
     return w
+
+
+# (projection, M, call count) of the README's LTX-Video benchmark table, in
+# its row order; the count-weighted total over these rows is its TOTAL row.
+PAGE_MICROBENCH = (
+    ("w2", 1400, 336), ("w1", 1400, 336), ("w2", 2450, 336), ("w1", 2450, 336),
+    ("w2", 5600, 480), ("w1", 5600, 480), ("w2", 9800, 144), ("w1", 9800, 144),
+    ("w2", 10850, 336), ("w1", 10850, 336), ("w2", 22400, 144), ("w1", 22400, 144),
+    ("w2", 43400, 144), ("w1", 43400, 144),
+)
+
+
+def page_workload(cfg: str, m: int, r: int) -> str:
+    k, n = (4096, 16384) if cfg == "w1" else (16384, 4096)
+    return f"page_{cfg}_m{m}_k{k}_n{n}_r{r}"
 
 
 WORKLOADS = _build_workloads()

@@ -268,3 +268,10 @@ def test_argument_errors_on_device():
         assert e.value.code == ll.LL_ERR_INVALID_ARG
     finally:
         d.close()
+
+
+@pytest.mark.parametrize("cfg,M,r", [("w1", 1400, 32), ("w2", 2450, 64), ("w1", 43400, 64), ("w2", 10850, 32)])
+def test_page_microbench_shapes_sampled(cfg, M, r):
+    """The README's LTX-Video FFN benchmark shapes (K / N read as 4096 <-> 16384)."""
+    from synth_inputs import page_workload
+    _sampled(page_workload(cfg, M, r))
