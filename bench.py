@@ -299,6 +299,72 @@ def run_page_suite(args):
     return 0
 
 
+def run_crossover_suite(args):
+    """Every kernel variant against the token count M at K = 4096,
+    N = 16384 and the given rank (the sweep's shape family): where the
+    streaming, small-tile and fused large-M kernels cross over, and what the
+    AUTO dispatch picks."""
+    import torch
+    import rank_fp8_residual_b200 as ll
+    from synth_inputs import make_weights
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    K, N, r = 4096, 16384, args.rank
+    B, A, Q, scale, bias = make_weights(K, N, r, seed=0)
+    layer = ll.LiteLinearLayer(N, K, r, SCALE_PER_ROW)
+    layer.set_weights(A.to(dev), B.to(dev), Q.to(dev), scale.to(dev), bias.to(dev))
+    h = layer.handle
+    steps = max(1, min(args.steps, 30))
+    variants = {"stream": ll.LL_VARIANT_STREAM, "small": ll.LL_VARIANT_SMALL, "tc": ll.LL_VARIANT_TC,
+                "tc_pair": ll.LL_VARIANT_TC_PAIR, "auto": ll.LL_VARIANT_AUTO}
+    points = []
+    for M in (1, 16, 32, 64, 96, 128, 192, 256, 384, 512, 1024, 2048, 4096):
+        ll.ll_reserve(h, M)
+        g = torch.Generator(device=dev)
+        g.manual_seed(2000 + M)
+        x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        row = {"M": M}
+        for name, v in variants.items():
+            if name == "stream" and M > 64:
+                continue  # the streaming kernel serves M <= 64 only
+            if name == "tc_pair" and M <= 64:
+                continue
+            ll.ll_set_variant(h, v)
+            ev = []
+            with torch.cuda.stream(stream):
+                for i in range(args.warmup + steps):
+                    flush.zero_()
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    ll.ll_forward(h, x, y, M, stream)
+                    b.record(stream)
+                    if i >= args.warmup:
+                        ev.append((a, b))
+            torch.cuda.synchronize()
+            st = ll.ll_status(h)
+            if st != ll.LL_OK:
+                raise SystemExit(f"device status: {ll.status_string(st)}")
+            us = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+            row[name] = round(us[len(us) // 2], 2)
+        timed = {k: v for k, v in row.items() if k not in ("M", "auto")}
+        row["fastest"] = min(timed, key=timed.get)
+        points.append(row)
+        del x, y
+    layer.close()
+    line = {"metric": "ll_forward time per variant against M", "value": None, "unit": "us",
+            "higher_is_better": False, "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"crossover_k{K}_n{N}_r{r}", "l2": "flushed between calls",
+                       "points": points}}
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -309,14 +375,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", default="auto", choices=["auto", "tc", "tc_pair", "small", "stream"],
                     help="kernel variant (auto picks by token count)")
-    ap.add_argument("--suite", default=None, choices=["page"],
-                    help="page: the README's LTX-Video FFN shapes, count-weighted total (one GPU)")
+    ap.add_argument("--suite", default=None, choices=["page", "crossover"],
+                    help="page: the README's LTX-Video FFN shapes, count-weighted total; "
+                         "crossover: every kernel variant against M (one GPU)")
     ap.add_argument("--rank", type=int, default=64, choices=[32, 64], help="rank of the --suite shapes")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.suite == "page":
         return run_page_suite(args)
+    if args.suite == "crossover":
+        return run_crossover_suite(args)
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
