@@ -22,7 +22,8 @@
 // fill the SMs in as few equal waves as possible).  Q is the MMA A operand:
 // eight converter warps widen the e4m3fn codes exactly to bf16 and store
 // them into TMEM stages of two K steps (64 columns); x is the B operand,
-// staged by TMA.  Persistent CTAs take tiles from a device-wide counter in a
+// staged by TMA, whose two chunks of a stage complete on that stage's TMEM
+// barrier, so the MMA issuer waits once per eight MMAs.  Persistent CTAs take tiles from a device-wide counter in a
 // grouped raster order (8 token tiles per group) so that the tiles in flight
 // share their x and Q slabs in L2.  Every tile, the first included, comes
 // from that counter.
@@ -129,7 +130,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     for (int s = 0; s < kTcSX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
     // A Q slot and a TMEM stage each hold one stage, which one team reads / writes.
     for (int s = 0; s < kTcSQ; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], kTcConvWarps / 2); }
-    for (int s = 0; s < kTcNA; ++s) { mbar_init(&a_full[s], kTcConvWarps / 2); mbar_init(&a_empty[s], 1); }
+    // a_full[stage]: the converter team's eight arrivals plus the x
+    // producer's (with the transaction bytes of the stage's two x chunks),
+    // so one wait tells the MMA issuer that both operands are in place.
+    for (int s = 0; s < kTcNA; ++s) { mbar_init(&a_full[s], kTcConvWarps / 2 + 1); mbar_init(&a_empty[s], 1); }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kTcEpiWarps);
     for (int s = 0; s < kTcTileRing; ++s) {
@@ -209,7 +213,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     if (lane == 0) {
       int xi = 0, ti = 0;
       uint32_t xph = 0, tph = 0;
-      long long nx = 0;
+      uint32_t lr_ph = 0;  // per-slot phase bits of x_full (used by the low-rank chunks only)
+      long long nx = 0;    // low-rank loads issued (on x_full)
+      long long gsx = 0;   // residual stages issued (on a_full)
+      long long pend_s = 0;  // residual stages whose loads were issued
       bool ok = true, waited_primary = false;
       const uint32_t x_bytes = static_cast<uint32_t>(bt) * kBK * 2u;
       const uint32_t a_bytes = 128u * klr * 2u;
@@ -223,12 +230,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
         if (p.withhold) { ok = false; break; }
         int f0, t0;
         tc_tile_coords(T, p.n_ftiles, p.n_ttiles, bt, f0, t0);
-        for (int kb = 0; kb < 2 * nS && ok; ++kb) {
-          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&x_full[xi], x_bytes);
-          tma_load_2d(sx + xi * kTcXSlot, &p.tm_x, &x_full[xi], kb * kBK, t0);
-          ++nx;
-          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+        // Residual stages: the two x chunks of stage s go into the next two
+        // slots and complete on the stage's a_full barrier.
+        for (int s = 0; s < nS && ok; ++s) {
+          int slot[2];
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+            slot[h] = xi;
+            if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          }
+          if (!ok) break;
+          uint64_t* bar = &a_full[gsx % kTcNA];
+          mbar_arrive_expect_tx(bar, 2 * x_bytes);
+          tma_load_2d(sx + slot[0] * kTcXSlot, &p.tm_x, bar, 2 * s * kBK, t0);
+          tma_load_2d(sx + slot[1] * kTcXSlot, &p.tm_x, bar, (2 * s + 1) * kBK, t0);
+          ++gsx;
+          pend_s = gsx;
         }
         if (ok && nR > 0 && !waited_primary && p.lr_from_primary) {
           pdl_wait_primary();
@@ -236,28 +253,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
         }
         for (int jb = 0; jb < nR && ok; ++jb) {
           // slot 1: A'_hi | A'_lo chunk; slot 2: t_hi chunk; slot 3: t_lo chunk
-          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&x_full[xi], 2 * a_bytes);
-          tma_load_2d(sx + xi * kTcXSlot, &p.tm_ahi, &x_full[xi], jb * klr, f0);
-          tma_load_2d(sx + xi * kTcXSlot + a_bytes, &p.tm_alo, &x_full[xi], jb * klr, f0);
-          ++nx;
-          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
-          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&x_full[xi], t_bytes);
-          tma_load_2d(sx + xi * kTcXSlot, &p.tm_thi, &x_full[xi], jb * klr, t0);
-          ++nx;
-          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
-          if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&x_full[xi], t_bytes);
-          tma_load_2d(sx + xi * kTcXSlot, &p.tm_tlo, &x_full[xi], jb * klr, t0);
-          ++nx;
-          if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          const CUtensorMap* maps[3] = {&p.tm_ahi, &p.tm_thi, &p.tm_tlo};
+          for (int w = 0; w < 3; ++w) {
+            if (!mbar_wait(&x_empty[xi], xph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+            uint64_t* bar = &x_full[xi];
+            if (w == 0) {
+              mbar_arrive_expect_tx(bar, 2 * a_bytes);
+              tma_load_2d(sx + xi * kTcXSlot, &p.tm_ahi, bar, jb * klr, f0);
+              tma_load_2d(sx + xi * kTcXSlot + a_bytes, &p.tm_alo, bar, jb * klr, f0);
+            } else {
+              mbar_arrive_expect_tx(bar, t_bytes);
+              tma_load_2d(sx + xi * kTcXSlot, maps[w], bar, jb * klr, t0);
+            }
+            ++nx;
+            lr_ph ^= 1u << xi;
+            if (++xi == kTcSX) { xi = 0; xph ^= 1; }
+          }
         }
         if (!ok) break;
       }
-      if (!ok) {
-        for (long long i = (nx > kTcSX ? nx - kTcSX : 0); i < nx; ++i)
-          mbar_wait_drain(&x_full[i % kTcSX], static_cast<uint32_t>((i / kTcSX) & 1), p.watch);
+      if (!ok && (pend_s > 0 || nx > 0)) {
+        // Loads already issued must land before the CTA exits.  Residual
+        // chunks complete on a_full, which also counts the converters (who
+        // may have left), so instead of waiting on it wait a bounded settle
+        // time, far above any load latency.
+        const uint64_t c0 = clock_cycles();
+        while (clock_cycles() - c0 < 400000ull) {  // >= 200 us at any clock up to 2 GHz
+        }
       }
     }
   } else if (warp == 1) {
@@ -265,6 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     if (lane == 0) {
       int xi = 0, ai = 0, ti = 0;
       uint32_t xph = 0, aph = 0, accph = 0, tph = 0;
+      uint32_t lr_ph = 0;  // per-slot phase bits of x_full (low-rank chunks only)
       bool ok = true;
       const uint32_t a_bytes = 128u * klr * 2u;
       for (;;) {
@@ -280,11 +303,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
         if (!mbar_wait(acc_empty, accph ^ 1, p.watch, kErrTimeoutMma)) break;
         tc_fence_after();
         for (int s = 0; s < nS && ok; ++s) {
+          // One wait per stage: converted Q (team) and both x chunks (TMA).
           if (!mbar_wait(&a_full[ai], aph, p.watch, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
-            if (!mbar_wait(&x_full[xi], xph, p.watch, kErrTimeoutMma)) { ok = false; break; }
-            tc_fence_after();
             const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sx + xi * kTcXSlot));
             const uint32_t at = tbase + kTcColA + ai * 64 + sub * 32;
 #pragma unroll
@@ -293,14 +316,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
             tc_commit(&x_empty[xi]);
             if (++xi == kTcSX) { xi = 0; xph ^= 1; }
           }
-          if (!ok) break;
           tc_commit(&a_empty[ai]);
           if (++ai == kTcNA) { ai = 0; aph ^= 1; }
         }
         for (int jb = 0; jb < nR && ok; ++jb) {
           int slot[3];
           for (int w = 0; w < 3; ++w) {
-            if (!mbar_wait(&x_full[xi], xph, p.watch, kErrTimeoutMma)) { ok = false; break; }
+            if (!mbar_wait(&x_full[xi], (lr_ph >> xi) & 1u, p.watch, kErrTimeoutMma)) { ok = false; break; }
+            lr_ph ^= 1u << xi;
             slot[w] = xi;
             if (++xi == kTcSX) { xi = 0; xph ^= 1; }
           }
