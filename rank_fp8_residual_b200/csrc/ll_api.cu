@@ -134,12 +134,14 @@ struct ll_layer {
   const void* c_x = nullptr;
   void* c_yptr = nullptr;
   int c_M = -1;
-  CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256, c_thik, c_tlok, c_x3;
+  CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256;
   CUtensorMap c_xs, c_this, c_tlos;  // streaming kernel: x and t boxes of Mt rows
   CUtensorMap tm_q3;  // 3-D view of the (row-cleared) residual, 4 K chunks per box
   CUtensorMap tm_q3b2;  // the same view, 2 K chunks per box (fused single-CTA kernel)
   CUtensorMap c_xbt, c_thibt, c_tlobt;  // fused single-CTA kernel: x and t boxes of bt rows
   int c_bt = 0;
+  CUtensorMap c_x2p, c_thip, c_tlop;  // CTA-pair kernel: x and t boxes of bt2 / 2 rows
+  int c_bt2 = 0;
   int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
   int variant = LL_VARIANT_AUTO;
   int withhold = 0;
@@ -274,9 +276,26 @@ int tc_tile_tokens(const ll_layer* h, int M) {
   return best;
 }
 
-// The CTA-pair kernel computes t with the warp-level kernel beside it.
-bool warp_lowrank(const ll_layer* h, int M) {
-  return choose_path(h, M) == PATH_TC2 && h->r_pad > 0 && h->r_pad <= 128;
+int pair_cluster_count(ll_layer* h);
+
+// Tokens per tile of the CTA-pair kernel (256 features per tile), by the
+// same model over the co-resident clusters; narrower tiles are allowed down
+// to 32 tokens for small M.
+int tc2_tile_tokens(ll_layer* h, int M) {
+  constexpr int kTileCost = 80;
+  const int n_fpairs = (h->N + 255) / 256;
+  const int clusters = pair_cluster_count(h);
+  int best = 256;
+  long long best_cost = -1;
+  for (int bt = 256; bt >= 32; bt -= 32) {
+    const long long tiles = static_cast<long long>(n_fpairs) * ((M + bt - 1) / bt);
+    const long long cost = (tiles + clusters - 1) / clusters * (bt + kTileCost);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bt;
+    }
+  }
+  return best;
 }
 
 struct LrPlan {
@@ -313,7 +332,7 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   // streaming kernel's tiles leave free.  The other kernels wait for it, so
   // it takes all SMs.
   int budget = h->num_sms;
-  if (path == PATH_TC1) budget = std::max(1, h->num_sms * 3 / 4);
+  if (path == PATH_TC1 || path == PATH_TC2) budget = std::max(1, h->num_sms * 3 / 4);
   if (path == PATH_STREAM) budget = std::max(1, h->num_sms - stream_ctas(h));
   int ks = std::max(1, budget / ctas);
   ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);
@@ -324,7 +343,6 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
 }
 
 size_t part_bytes_for(const ll_layer* h, int M) {
-  if (warp_lowrank(h, M)) return 0;
   const LrPlan p = plan_lowrank(h, M);
   return p.ksplit > 1 ? static_cast<size_t>(p.ksplit) * M * h->r_pad * sizeof(float) : 0;
 }
@@ -336,8 +354,6 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   ok &= make_map(&h->c_x128, x, kBF16, M, h->K, 2ull * h->K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&h->c_x256, x, kBF16, M, h->K, 2ull * h->K, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&h->c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (h->K % 64 == 0) ok &= make_map3(&h->c_x3, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, 128, 2,
-                                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (M > 128) {
     const int bt = tc_tile_tokens(h, M);
     h->c_bt = bt;
@@ -346,6 +362,20 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
       const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
       ok &= make_map(&h->c_thibt, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
       ok &= make_map(&h->c_tlobt, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
+    }
+  }
+  if (choose_path(h, M) == PATH_TC2) {
+    const int bt2 = tc2_tile_tokens(h, M);
+    const uint32_t hb = static_cast<uint32_t>(bt2 / 2);
+    h->c_bt2 = bt2;
+    if (h->K % 64 == 0)
+      ok &= make_map3(&h->c_x2p, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, hb, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+      ok &= make_map(&h->c_x2p, x, kBF16, M, h->K, 2ull * h->K, kBK, hb, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (h->r_pad > 0) {
+      const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+      ok &= make_map(&h->c_thip, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, hb, sw);
+      ok &= make_map(&h->c_tlop, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, hb, sw);
     }
   }
   if (M <= kStreamMaxM) {
@@ -365,8 +395,6 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
     ok &= make_map(&h->c_tlo128, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&h->c_thi256, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
     ok &= make_map(&h->c_tlo256, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
-    ok &= make_map(&h->c_thik, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
-    ok &= make_map(&h->c_tlok, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
   }
   if (!ok) {
     h->c_M = -1;
@@ -376,14 +404,6 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   h->c_yptr = y;
   h->c_M = M;
   return true;
-}
-
-int launch_warp_lowrank(ll_layer* h, const void* x, int M, cudaStream_t st) {
-  using namespace llk;
-  dim3 grid((M + 15) / 16, h->r_pad / 32);
-  ll_lrdown_warp_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(x), h->B, h->t_hi, h->t_lo, M, h->K,
-                                              h->r_pad);
-  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
 
 int pair_cluster_count(ll_layer* h) {
@@ -405,10 +425,8 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   using namespace llk;
   h->last_launches = 0;
   const Path path = choose_path(h, M);
-  const bool wlr = warp_lowrank(h, M);
   const LrPlan lp = plan_lowrank(h, M);
-  const size_t part_need =
-      (!wlr && lp.ksplit > 1) ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0;
+  const size_t part_need = lp.ksplit > 1 ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0;
   int rc = ensure_workspace(h, M, st, part_need);
   if (rc != LL_OK) return rc;
   if (!build_call_maps(h, x, y, M)) return LL_ERR_CUDA;
@@ -422,12 +440,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     cudaEventRecord(h->ev[0], st);
   }
 
-  if (wlr) {
-    rc = launch_warp_lowrank(h, x, M, st);
-    if (rc != LL_OK) return rc;
-    h->names[launches++] = "ll_lrdown_warp_kernel";
-    if (prof) cudaEventRecord(h->ev[launches], st);
-  } else if (h->r_pad > 0) {
+  if (h->r_pad > 0) {
     if (lp.rc != h->b_box) {
       if (!make_map(&h->tm_b, h->B, kBF16, h->r_pad, h->K, 2ull * h->K, kBK, lp.rc, CU_TENSOR_MAP_SWIZZLE_128B))
         return LL_ERR_CUDA;
@@ -455,9 +468,8 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
   }
 
-  // Programmatic overlap with the kernel that produces t, where the main
-  // kernel's schedule tolerates SMs that start late.
-  const bool overlap = h->r_pad > 0 && !prof && (path != PATH_TC2 || wlr);
+  // Programmatic overlap with the kernel that produces t.
+  const bool overlap = h->r_pad > 0 && !prof;
   cudaLaunchConfig_t cfg = {};
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -495,14 +507,12 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   } else if (path == PATH_TC2) {
     Tc2Params tp;
     tp.dims3 = h->K % 64 == 0 ? 1 : 0;
-    tp.tm_x = tp.dims3 ? h->c_x3 : h->c_x128;
-    tp.tm_q = tp.dims3 ? h->tm_q3 : h->tm_qf;
-    tp.xc = tp.dims3 ? 2 : 1;
-    tp.qc = tp.dims3 ? 4 : 1;
+    tp.tm_x = h->c_x2p;
+    tp.tm_q = tp.dims3 ? h->tm_q3b2 : h->tm_qf;
     tp.tm_ahi = h->tm_ahi;
     tp.tm_alo = h->tm_alo;
-    tp.tm_thi = h->c_thik;
-    tp.tm_tlo = h->c_tlok;
+    tp.tm_thi = h->c_thip;
+    tp.tm_tlo = h->c_tlop;
     tp.tm_y = h->c_y;
     tp.scale = h->scale_eff;
     tp.bias = h->has_bias ? h->bias : nullptr;
@@ -511,12 +521,12 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     tp.K = h->K;
     tp.r_pad = h->r_pad;
     tp.klr = h->klr;
+    tp.bt = h->c_bt2;
     tp.n_fpairs = (h->N + 255) / 256;
-    tp.m32 = (M + 31) / 32 * 32;
-    const long long units = static_cast<long long>(tp.n_fpairs) * tp.m32;
-    const int max_clusters = pair_cluster_count(h);
-    const int clusters = static_cast<int>(std::max<long long>(1, std::min<long long>(max_clusters, (units + 255) / 256)));
-    tp.seg = static_cast<int>(((units + clusters - 1) / clusters + 31) / 32 * 32);
+    tp.n_ttiles = (M + tp.bt - 1) / tp.bt;
+    tp.sched = h->sched;
+    const int tiles = tp.n_fpairs * tp.n_ttiles;
+    const int clusters = std::max(1, std::min(pair_cluster_count(h), tiles));
     tp.lr_from_primary = overlap ? 1 : 0;
     tp.withhold = h->withhold;
     tp.watch = watch;
@@ -887,6 +897,7 @@ int ll_set_variant(ll_handle h, int variant) {
              variant != LL_VARIANT_TC_PAIR && variant != LL_VARIANT_STREAM))
     return fail(LL_ERR_INVALID_ARG);
   h->variant = variant;
+  h->c_M = -1;  // the per-call tensor maps depend on the kernel chosen
   return LL_OK;
 }
 
