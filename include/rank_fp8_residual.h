@@ -175,11 +175,11 @@ const char *ll_kernel_name(ll_handle h, int i);
  * synchronisation.  Such a caller cannot use ll_create (it copies the
  * factors into library-owned memory) or ll_forward (it grows a workspace
  * on demand).  This call takes no handle: the caller passes every input
- * and the output, and the intermediate t = x B^T (bf16 hi + lo), its
- * split-K partial sums and arrival counters, a device status word and,
- * for a per-tensor scale, the scale broadcast to N rows live in one static
- * device array of LL_NOALLOC_SCRATCH_BYTES.  Every GPU on which the library's device code
- * is loaded holds that array until the process exits.
+ * and the output, and the intermediate t = x B^T (bf16 hi + lo), a device
+ * status word and, for a per-tensor scale, the scale broadcast to N rows
+ * live in one static device array of LL_NOALLOC_SCRATCH_BYTES.  Every GPU
+ * on which the library's device code is loaded holds that array until the
+ * process exits.
  *
  * y is the forward of ll_forward with the SMALL variant (residual and
  * low-rank terms in separate accumulators, A used as given) and meets the
@@ -196,9 +196,7 @@ const char *ll_kernel_name(ll_handle h, int i);
  *     256 + 4 * M * r32 bytes  (+ 4 * N rounded up to 256 for a per-tensor
  *     scale), at most LL_NOALLOC_SCRATCH_BYTES.
  * A larger request returns LL_ERR_SCRATCH_LIMIT and launches nothing
- * (e.g. r = 512 allows M up to 8191, r = 64 up to 65535).  Split-K
- * partials only use what is left over; when little is, the down-projection
- * runs with fewer splits.
+ * (e.g. r = 512 allows M up to 8191, r = 64 up to 65535).
  *
  * Not checked here: the weights are read as given on every call, with no
  * scan for NaN codes or non-finite scales (ll_set_weights does those
@@ -206,8 +204,7 @@ const char *ll_kernel_name(ll_handle h, int i);
  *
  * Shared scratch: every call on a device uses the same array, and the
  * array keeps the last call's contents.  Each call clears the status word
- * and fully rewrites t before reading it; the split-K counters start at
- * zero when the library loads and every call leaves them at zero.  Calls whose kernels overlap on
+ * and fully rewrites t before reading it.  Calls whose kernels overlap on
  * the GPU (issued on two streams without ordering, or from two host
  * threads) race on the array and give wrong results: order them on one
  * stream or with events.

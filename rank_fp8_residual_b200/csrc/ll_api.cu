@@ -98,6 +98,12 @@ int next_pow2_ge32(int v) {
 
 }  // namespace
 
+// Joint plan of the single-CTA fused kernel and the down-projection.
+struct TcChoice {
+  int bt;  // tokens per fused-kernel tile
+  int ks;  // K splits of the down-projection (1 when r == 0)
+};
+
 struct ll_layer {
   int N = 0, K = 0, r = 0, r_pad = 0, klr = 64, scale_mode = 0;
   int device = 0, num_sms = 0;
@@ -116,13 +122,10 @@ struct ll_layer {
   int* status = nullptr;      // device status word
   int* flags = nullptr;       // [2] set-time scan flags
   int* sched = nullptr;       // [2] tile scheduler of the fused kernel
-  int* lr_cnt = nullptr;      // [kLrMaxTiles] split-K arrival counters of the down-projection
   // workspace for t
   int ws_M = 0;
   uint16_t* t_hi = nullptr;
   uint16_t* t_lo = nullptr;
-  float* part = nullptr;
-  size_t part_bytes = 0;
   // host-buffer forward staging
   void* dx = nullptr;
   void* dy = nullptr;
@@ -140,6 +143,8 @@ struct ll_layer {
   CUtensorMap tm_q3b2;  // the same view, 2 K chunks per box (fused single-CTA kernel)
   CUtensorMap c_xbt, c_thibt, c_tlobt;  // fused single-CTA kernel: x and t boxes of bt rows
   int c_bt = 0;
+  mutable int tcp_M = -1;  // M of the cached joint plan
+  mutable TcChoice tcp{};
   CUtensorMap c_x2p, c_thip, c_tlop;  // CTA-pair kernel: x and t boxes of bt2 / 2 rows
   int c_bt2 = 0;
   int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
@@ -171,10 +176,8 @@ void free_layer_mem(ll_layer* h) {
   cudaFree(h->status);
   cudaFree(h->flags);
   cudaFree(h->sched);
-  cudaFree(h->lr_cnt);
   cudaFree(h->t_hi);
   cudaFree(h->t_lo);
-  cudaFree(h->part);
   cudaFree(h->dx);
   cudaFree(h->dy);
 }
@@ -203,9 +206,8 @@ int set_smem_attrs_once() {
   return rc;
 }
 
-// Grow the t workspace to hold `M` rows and the split partials to
-// `part_need` bytes (stream-ordered).
-int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
+// Grow the t workspace to hold `M` rows (stream-ordered).
+int ensure_workspace(ll_layer* h, int M, cudaStream_t st) {
   if (h->r_pad == 0) return LL_OK;
   if (M > h->ws_M) {
     int newM = std::max(M, h->ws_M * 3 / 2);
@@ -224,17 +226,6 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st, size_t part_need) {
     h->t_lo = tl;
     h->ws_M = newM;
     h->c_M = -1;  // maps over t must be rebuilt
-  }
-  if (part_need > h->part_bytes) {
-    float* pp = nullptr;
-    const size_t nb = std::max(part_need, h->part_bytes * 3 / 2);
-    if (cudaMallocAsync(reinterpret_cast<void**>(&pp), nb, st) != cudaSuccess) {
-      cudaGetLastError();
-      return LL_ERR_OOM;
-    }
-    if (h->part) cudaFreeAsync(h->part, st);
-    h->part = pp;
-    h->part_bytes = nb;
   }
   return LL_OK;
 }
@@ -255,26 +246,80 @@ Path choose_path(const ll_layer* h, int M) {
 // CTAs of the streaming kernel: one per 128-feature tile, at most one per SM.
 int stream_ctas(const ll_layer* h) { return std::min((h->N + 127) / 128, h->num_sms); }
 
-// Tokens per tile of the single-CTA fused kernel: the multiple of 32 up to
-// 256 that finishes the tiles in the least time per SM, modelled as waves
-// of num_sms tiles times (tile width + a fixed per-tile cost worth about 80
-// token columns: the epilogue and the pipeline fill); ties go to the wider
-// tile.
-int tc_tile_tokens(const ll_layer* h, int M) {
-  constexpr int kTileCost = 80;
+// Joint plan of the single-CTA fused kernel and the down-projection beside
+// it.  The down-projection's CTAs hold their SMs until t is written, so the
+// fused kernel's CTAs on those SMs start late and (taking tiles from a
+// shared counter) take fewer tiles.  The plan picks the tile width (a
+// multiple of 32 from 128 to 256) and the number of K splits of the
+// down-projection that minimise a model of the finishing time: tiles of
+// equal duration handed out greedily to the SMs free at time 0 and to the
+// down-projection's SMs once it ends.  The model's rates are fitted to
+// forward times measured on B200 (they rank plans; they are not a
+// prediction of the time).
+double tc_finish_us(long long tiles, int sms, int late, double t_tile, double t_lr) {
+  const int early = sms - late;
+  // A tile's low-rank step needs t: early tiles cannot end before it is there.
+  const double d0 = std::max(0.0, t_lr + 1.0 - t_tile);
+  long long done = 0;
+  long long ke = 0, kl = 0;
+  for (;;) {
+    const double se = early > 0 ? d0 + ke * t_tile : 1e30;
+    const double sl = late > 0 ? t_lr + kl * t_tile : 1e30;
+    double s;
+    if (se <= sl) {
+      done += early;
+      s = se;
+      ++ke;
+    } else {
+      done += late;
+      s = sl;
+      ++kl;
+    }
+    if (done >= tiles) return s + t_tile;
+  }
+}
+
+TcChoice plan_tc1(const ll_layer* h, int M) {
+  if (h->tcp_M == M) return h->tcp;
+  constexpr double kStageNsPerToken = 2.8;  // per 2-K-step stage and (bt + 32) tokens
+  constexpr double kTileFixedUs = 2.5;      // pipeline fill + epilogue per tile
+  constexpr double kLrFixedUs = 3.5;        // down-projection launch, first loads, reduction
+  constexpr double kLrCtaGBs = 70.0;        // x read rate of one down-projection CTA
+  constexpr double kLrMaxGBs = 5500.0;      // and of all of them together
+  const int nK = (h->K + llk::kBK - 1) / llk::kBK;
+  const int nS = (nK + 1) / 2;
   const int n_ftiles = (h->N + 127) / 128;
-  int best = 256;
-  long long best_cost = -1;
+  const int m_tiles = (M + 127) / 128;
+  const int rc = std::min(std::max(h->r_pad, 32), 256);
+  const int r_chunks = h->r_pad > 0 ? (h->r_pad + rc - 1) / rc : 0;
+  const double x_mb = 2.0 * M * h->K * r_chunks / 1e6;
+  TcChoice best{256, 1};
+  double best_t = -1;
   for (int bt = 256; bt >= 128; bt -= 32) {
     const long long tiles = static_cast<long long>(n_ftiles) * ((M + bt - 1) / bt);
-    const long long cost = (tiles + h->num_sms - 1) / h->num_sms * (bt + kTileCost);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = bt;
+    const double t_tile = kTileFixedUs + 0.3 * h->r_pad / 32 + nS * (bt + 32) * kStageNsPerToken * 1e-3;
+    const int ks_max = h->r_pad > 0 ? std::min(nK, llk::kLrMaxSplit) : 1;
+    for (int ks = 1; ks <= ks_max; ++ks) {
+      const int lr_ctas = h->r_pad > 0 ? m_tiles * r_chunks * ks : 0;
+      if (ks > 1 && lr_ctas > h->num_sms) break;
+      const int late = std::min(lr_ctas, h->num_sms);
+      const double t_lr =
+          h->r_pad > 0 ? kLrFixedUs + x_mb / std::min(late * kLrCtaGBs, kLrMaxGBs) * 1e3 : 0.0;
+      const double t = tc_finish_us(tiles, h->num_sms, late, t_tile, t_lr);
+      // A wider tile or fewer down-projection CTAs unless the model gains
+      // more than 1 %.
+      if (best_t < 0 || t < best_t * 0.99) {
+        best_t = t;
+        best = TcChoice{bt, ks};
+      }
     }
   }
+  h->tcp_M = M;
+  h->tcp = best;
   return best;
 }
+
+int tc_tile_tokens(const ll_layer* h, int M) { return plan_tc1(h, M).bt; }
 
 int pair_cluster_count(ll_layer* h);
 
@@ -324,27 +369,37 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   p.r_chunks = (h->r_pad + p.rc - 1) / p.rc;
   p.tmem_cols = next_pow2_ge32(p.rc);
   const int ctas = p.m_tiles * p.r_chunks;
-  // With the single-CTA fused kernel the down-projection runs beside it on
-  // a quarter of the SMs; the other kernels wait for it, so it takes all.
-  // The down-projection runs beside the fused kernels: on three quarters of
-  // the SMs next to the large-M kernel (whose CTAs take tiles from a shared
-  // counter, so those that start late take fewer), and on the SMs the
-  // streaming kernel's tiles leave free.  The other kernels wait for it, so
-  // it takes all SMs.
+  // The down-projection runs beside the fused kernels: as many splits as
+  // the joint plan gives next to the single-CTA kernel, three quarters of
+  // the SMs next to the CTA-pair kernel, and the SMs the streaming
+  // kernel's tiles leave free.  The other kernels wait for it, so it takes
+  // all SMs.
   int budget = h->num_sms;
-  if (path == PATH_TC1 || path == PATH_TC2) budget = std::max(1, h->num_sms * 3 / 4);
+  if (path == PATH_TC2) budget = std::max(1, h->num_sms * 3 / 4);
   if (path == PATH_STREAM) budget = std::max(1, h->num_sms - stream_ctas(h));
   int ks = std::max(1, budget / ctas);
   ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);
-  if (ctas > llk::kLrMaxTiles) ks = 1;
+  if (path == PATH_TC1 && M > 128) ks = plan_tc1(h, M).ks;
   p.kb_per_split = (nK + ks - 1) / ks;
   p.ksplit = (nK + p.kb_per_split - 1) / p.kb_per_split;
   return p;
 }
 
-size_t part_bytes_for(const ll_layer* h, int M) {
-  const LrPlan p = plan_lowrank(h, M);
-  return p.ksplit > 1 ? static_cast<size_t>(p.ksplit) * M * h->r_pad * sizeof(float) : 0;
+// Launches the down-projection; its K splits form one cluster per tile.
+cudaError_t launch_lrdown(const llk::LrDownParams& lpp, const LrPlan& lp, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(lp.m_tiles, lp.r_chunks, lp.ksplit);
+  cfg.blockDim = dim3(llk::kLrThreads);
+  cfg.dynamicSmemBytes = llk::lr_smem_bytes(lp.rc);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(lp.ksplit);
+  cfg.attrs = attr;
+  cfg.numAttrs = lp.ksplit > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, llk::ll_lrdown_kernel, lpp);
 }
 
 bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
@@ -426,8 +481,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   h->last_launches = 0;
   const Path path = choose_path(h, M);
   const LrPlan lp = plan_lowrank(h, M);
-  const size_t part_need = lp.ksplit > 1 ? static_cast<size_t>(lp.ksplit) * M * h->r_pad * sizeof(float) : 0;
-  int rc = ensure_workspace(h, M, st, part_need);
+  int rc = ensure_workspace(h, M, st);
   if (rc != LL_OK) return rc;
   if (!build_call_maps(h, x, y, M)) return LL_ERR_CUDA;
   const Watch watch{h->status, h->timeout_ns};
@@ -451,8 +505,6 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     lpp.tm_b = h->tm_b;
     lpp.t_hi = h->t_hi;
     lpp.t_lo = h->t_lo;
-    lpp.part = h->part;
-    lpp.cnt = h->lr_cnt;
     lpp.M = M;
     lpp.K = h->K;
     lpp.r_pad = h->r_pad;
@@ -461,11 +513,13 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     lpp.ksplit = lp.ksplit;
     lpp.kb_per_split = lp.kb_per_split;
     lpp.watch = watch;
-    dim3 grid(lp.m_tiles, lp.r_chunks, lp.ksplit);
-    ll_lrdown_kernel<<<grid, kLrThreads, lr_smem_bytes(lp.rc), st>>>(lpp);
+    const cudaError_t lerr = launch_lrdown(lpp, lp, st);
     h->names[launches++] = "ll_lrdown_kernel";
     if (prof) cudaEventRecord(h->ev[launches], st);
-    if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
+    if (lerr != cudaSuccess) {
+      cudaGetLastError();
+      return LL_ERR_CUDA;
+    }
   }
 
   // Programmatic overlap with the kernel that produces t.
@@ -675,7 +729,6 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
   ok &= cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
   ok &= cudaMalloc(&h->flags, 2 * sizeof(int)) == cudaSuccess;
   ok &= cudaMalloc(&h->sched, 2 * sizeof(int)) == cudaSuccess;
-  ok &= cudaMalloc(&h->lr_cnt, llk::kLrMaxTiles * sizeof(int)) == cudaSuccess;
   if (h->r_pad > 0) {
     ok &= cudaMalloc(&h->A, sizeof(uint16_t) * nrp) == cudaSuccess;
     ok &= cudaMalloc(&h->Ahi, sizeof(uint16_t) * nrp) == cudaSuccess;
@@ -692,7 +745,6 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
   h->Qf = h->Q;
   cudaMemset(h->status, 0, sizeof(int));
   cudaMemset(h->sched, 0, 2 * sizeof(int));
-  cudaMemset(h->lr_cnt, 0, llk::kLrMaxTiles * sizeof(int));
   using namespace llk;
   ok &= make_map(&h->tm_q, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_64B);
   h->tm_qf = h->tm_q;
@@ -880,10 +932,7 @@ int ll_forward_host(ll_handle h, const void* x_host, void* y_host, int M, void* 
 int ll_reserve(ll_handle h, int max_M) {
   g_last_error = LL_OK;
   if (!h || max_M < 0) return fail(LL_ERR_INVALID_ARG);
-  // The partial-sum buffer is largest at the biggest M of each tile count.
-  size_t need = 0;
-  for (int m = 128; m - 128 < max_M; m += 128) need = std::max(need, part_bytes_for(h, std::min(m, max_M)));
-  int rc = ensure_workspace(h, max_M, 0, need);
+  int rc = ensure_workspace(h, max_M, 0);
   if (cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     rc = LL_ERR_CUDA;
@@ -911,11 +960,9 @@ int ll_status(ll_handle h) {
     return fail(LL_ERR_CUDA);
   }
   if (v != 0) {
-    // A kernel gave up part-way: clear the status, the tile scheduler and
-    // the split-K counters.
+    // A kernel gave up part-way: clear the status and the tile scheduler.
     cudaMemset(h->status, 0, sizeof(int));
     cudaMemset(h->sched, 0, 2 * sizeof(int));
-    cudaMemset(h->lr_cnt, 0, llk::kLrMaxTiles * sizeof(int));
     cudaDeviceSynchronize();
     return LL_ERR_DEVICE_TIMEOUT;
   }
@@ -1046,10 +1093,8 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   NoAllocDevice* d = noalloc_setup(dev, &rc);
   if (!d) return rc;
 
-  // Scratch layout: status word (bytes 0-3) and split-K arrival counters
-  // (bytes 64-255, kept at zero between calls) | broadcast scale
-  // (per-tensor only) | t_hi [M, r_pad] | t_lo [M, r_pad] | split-K
-  // partials (what is left).
+  // Scratch layout: status word (bytes 0-3; 256 bytes reserved) |
+  // broadcast scale (per-tensor only) | t_hi [M, r_pad] | t_lo [M, r_pad].
   const int r_pad = (r + 31) / 32 * 32;
   const size_t t_bytes = static_cast<size_t>(M) * r_pad * sizeof(uint16_t);
   size_t off = 256;
@@ -1057,21 +1102,16 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   if (scale_mode == LL_SCALE_PER_TENSOR) off += round_up256(static_cast<size_t>(N) * sizeof(float));
   const size_t thi_off = off;
   const size_t tlo_off = thi_off + t_bytes;
-  const size_t part_off = tlo_off + t_bytes;  // 64-byte aligned: t rows are 64-byte multiples
-  if (part_off > LL_NOALLOC_SCRATCH_BYTES) return LL_ERR_SCRATCH_LIMIT;
+  if (tlo_off + t_bytes > LL_NOALLOC_SCRATCH_BYTES) return LL_ERR_SCRATCH_LIMIT;
 
   unsigned char* base = d->scratch;
   int* status = reinterpret_cast<int*>(base);
-  int* lr_cnt = reinterpret_cast<int*>(base + 64);
-  constexpr int kCounters = (256 - 64) / static_cast<int>(sizeof(int));
   const float* scale_n = scale;
   if (scale_mode == LL_SCALE_PER_TENSOR) scale_n = reinterpret_cast<float*>(base + scale_off);
   uint16_t* t_hi = reinterpret_cast<uint16_t*>(base + thi_off);
   uint16_t* t_lo = reinterpret_cast<uint16_t*>(base + tlo_off);
-  float* part = reinterpret_cast<float*>(base + part_off);
 
-  // Down-projection plan of the SMALL path, with the number of K splits
-  // cut to what the remaining scratch holds.
+  // Down-projection plan of the SMALL path.
   ll_layer view;
   view.N = N;
   view.K = K;
@@ -1079,21 +1119,7 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   view.r_pad = r_pad;
   view.num_sms = d->num_sms;
   view.variant = LL_VARIANT_SMALL;
-  LrPlan lp = plan_lowrank(&view, M);
-  if (lp.ksplit > 1 && lp.m_tiles * lp.r_chunks > kCounters) {
-    lp.kb_per_split = (K + kBK - 1) / kBK;
-    lp.ksplit = 1;
-  }
-  if (r_pad > 0 && lp.ksplit > 1) {
-    const size_t per_split = static_cast<size_t>(M) * r_pad * sizeof(float);
-    const size_t fit = (LL_NOALLOC_SCRATCH_BYTES - part_off) / per_split;
-    if (fit < static_cast<size_t>(lp.ksplit)) {
-      const int nK = (K + kBK - 1) / kBK;
-      const int ks = fit < 2 ? 1 : static_cast<int>(fit);
-      lp.kb_per_split = (nK + ks - 1) / ks;
-      lp.ksplit = (nK + lp.kb_per_split - 1) / lp.kb_per_split;
-    }
-  }
+  const LrPlan lp = plan_lowrank(&view, M);
 
   // Tensor maps over the caller's buffers; rank columns / rows past r read
   // as zeros (TMA fill), which stands in for the zero padding to r_pad.
@@ -1128,8 +1154,6 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
     lpp.tm_b = tm_b;
     lpp.t_hi = t_hi;
     lpp.t_lo = t_lo;
-    lpp.part = part;
-    lpp.cnt = lr_cnt;
     lpp.M = M;
     lpp.K = K;
     lpp.r_pad = r_pad;
@@ -1138,8 +1162,10 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
     lpp.ksplit = lp.ksplit;
     lpp.kb_per_split = lp.kb_per_split;
     lpp.watch = watch;
-    dim3 grid(lp.m_tiles, lp.r_chunks, lp.ksplit);
-    ll_lrdown_kernel<<<grid, kLrThreads, lr_smem_bytes(lp.rc), st>>>(lpp);
+    if (launch_lrdown(lpp, lp, st) != cudaSuccess) {
+      cudaGetLastError();
+      return LL_ERR_CUDA;
+    }
   }
   if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
 

@@ -12,8 +12,9 @@
 //   1. ll_lrdown_kernel   t = x B^T with tcgen05, fp32 accumulate in TMEM,
 //                         written as a bf16 pair (t_hi = bf16(t),
 //                         t_lo = bf16(t - t_hi)).  With several K splits
-//                         each CTA writes an fp32 partial sum and the last
-//                         CTA of a tile adds them in split order.
+//                         the splits of a tile form one cluster and add
+//                         their partial sums in split order over
+//                         distributed shared memory.
 //   2. ll_main_kernel     persistent fused GEMM.  Tile = 128 output
 //                         features x up to 128 tokens.  Q (e4m3fn) is the
 //                         MMA A operand: converter warps widen it exactly to
@@ -70,12 +71,10 @@ struct LrDownParams {
   CUtensorMap tm_b;  // bf16 [r_pad, K]  box {64, rc},  128B swizzle
   uint16_t* t_hi;    // [M, r_pad] bf16 bits
   uint16_t* t_lo;    // [M, r_pad]
-  float* part;       // [ksplit, M, r_pad] fp32 (ksplit > 1)
-  int* cnt;          // [gridDim.x * gridDim.y] arrival counters, zero between calls (ksplit > 1)
   int M, K, r_pad;
   int rc;            // box height of B = column block of t per CTA (<= 256)
   int tmem_cols;     // power of two >= rc
-  int ksplit;        // number of K splits (gridDim.z)
+  int ksplit;        // number of K splits (gridDim.z; one cluster along z when > 1)
   int kb_per_split;  // 64-wide K steps per split
   Watch watch;
 };
@@ -85,14 +84,20 @@ struct LrDownParams {
 constexpr int kLrMaxStages = 8;
 constexpr int kLrRingBytes = 192 * 1024;
 constexpr int kLrThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
-constexpr int kLrMaxSplit = 8;   // K splits per tile (the last CTA of a tile sums them)
-constexpr int kLrMaxTiles = 1024;  // tiles with split K (arrival counters)
+constexpr int kLrMaxSplit = 8;   // K splits per tile = CTAs per cluster (portable limit)
 
 __host__ __device__ constexpr int lr_stage_bytes(int rc) { return 128 * kBK * 2 + rc * kBK * 2; }
 __host__ __device__ constexpr int lr_stages(int rc) {
   return kLrRingBytes / lr_stage_bytes(rc) < kLrMaxStages ? kLrRingBytes / lr_stage_bytes(rc) : kLrMaxStages;
 }
 __host__ constexpr int lr_smem_bytes(int rc) { return lr_stages(rc) * lr_stage_bytes(rc) + 1024 + 256; }
+
+// Position of float4 column c4 of partial-sum row `row` in shared memory:
+// rows of rc fp32, the eight float4 of each 32-column block permuted by
+// row so that a warp's 32 rows store without bank conflicts.
+__device__ __forceinline__ uint32_t lr_part_off(int row, int c4, int rc) {
+  return static_cast<uint32_t>(row * rc * 4 + (((c4 & ~7) | ((c4 ^ row) & 7)) << 4));
+}
 
 __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_constant__ LrDownParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -109,12 +114,16 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
   const int m0 = blockIdx.x * 128;
   const int j0 = blockIdx.y * p.rc;
   const int wcols = min(p.rc, p.r_pad - j0);  // columns of t this CTA owns (multiple of 32)
-  const int kz = blockIdx.z;
+  const int kz = blockIdx.z;                  // K split = rank in the cluster
   const int nK = (p.K + kBK - 1) / kBK;
   const int kb_begin = kz * p.kb_per_split;
   const int kb_end = min(nK, kb_begin + p.kb_per_split);
   const int ncols = p.tmem_cols;
 
+  // Producer state (thread 0): the first lap of the ring is issued before
+  // the TMEM allocation and the block barrier.
+  int ps = 0, issued = 0;
+  uint32_t pph = 0;
   if (threadIdx.x == 0) {
     pdl_launch_dependents();
     for (int s = 0; s < n_stages; ++s) {
@@ -124,8 +133,14 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&p.tm_x);
-    tma_prefetch_desc(&p.tm_b);
+    for (int kb = kb_begin; kb < kb_end && issued < n_stages; ++kb, ++issued) {
+      uint8_t* st = smem + issued * stage_bytes;
+      mbar_arrive_expect_tx(&full[issued], stage_bytes);
+      tma_load_2d(st, &p.tm_x, &full[issued], kb * kBK, m0);
+      tma_load_2d(st + 128 * kBK * 2, &p.tm_b, &full[issued], kb * kBK, j0);
+    }
+    ps = issued % n_stages;
+    pph = issued == n_stages ? 1u : 0u;
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, ncols);
@@ -138,18 +153,15 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
 
   if (warp == 0) {
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      int issued = 0;
       bool ok = true;
-      for (int kb = kb_begin; kb < kb_end; ++kb) {
-        if (!mbar_wait(&empty[s], ph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
-        uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&full[s], stage_bytes);
-        tma_load_2d(st, &p.tm_x, &full[s], kb * kBK, m0);
-        tma_load_2d(st + 128 * kBK * 2, &p.tm_b, &full[s], kb * kBK, j0);
+      for (int kb = kb_begin + issued; kb < kb_end; ++kb) {
+        if (!mbar_wait(&empty[ps], pph ^ 1, p.watch, kErrTimeoutProducer)) { ok = false; break; }
+        uint8_t* st = smem + ps * stage_bytes;
+        mbar_arrive_expect_tx(&full[ps], stage_bytes);
+        tma_load_2d(st, &p.tm_x, &full[ps], kb * kBK, m0);
+        tma_load_2d(st + 128 * kBK * 2, &p.tm_b, &full[ps], kb * kBK, j0);
         ++issued;
-        if (++s == n_stages) { s = 0; ph ^= 1; }
+        if (++ps == n_stages) { ps = 0; pph ^= 1; }
       }
       if (!ok) {
         // Let every load already issued land before the CTA can exit.
@@ -183,50 +195,49 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
       mbar_wait_drain(drain, 0, p.watch);
     }
   } else {
-    // Epilogue: TMEM lane = token row.
+    // Epilogue: TMEM lane = token row.  One split: the bf16 pair straight to
+    // global memory.  Several: this split's fp32 partial into this CTA's
+    // shared memory (the ring is idle once every MMA is done).
     const int q = warp & 3;
-    const int m = m0 + 32 * q + lane;
+    const int row = 32 * q + lane;
+    const int m = m0 + row;
     if (__all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.watch, kErrTimeoutEpilogue))) {
       tc_fence_after();
       const bool empty_range = kb_end <= kb_begin;
       for (int c = 0; c < wcols; c += 32) {
         uint32_t v[32];
         tmem_ld32_wait(tbase + ((32u * q) << 16) + c, v);
-        if (m < p.M) {
-          if (p.ksplit == 1) {
-            uint32_t hi[16], lo[16];
+        if (empty_range) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float a = empty_range ? 0.f : __uint_as_float(v[2 * i]);
-              const float b = empty_range ? 0.f : __uint_as_float(v[2 * i + 1]);
-              const uint16_t ha = to_bf16_bits(a), hb = to_bf16_bits(b);
-              hi[i] = static_cast<uint32_t>(ha) | (static_cast<uint32_t>(hb) << 16);
-              lo[i] = pack_bf16x2(a - bf16_bits_to_float(ha), b - bf16_bits_to_float(hb));
-            }
-            uint4* dh = reinterpret_cast<uint4*>(p.t_hi + static_cast<size_t>(m) * p.r_pad + j0 + c);
-            uint4* dl = reinterpret_cast<uint4*>(p.t_lo + static_cast<size_t>(m) * p.r_pad + j0 + c);
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (p.ksplit > 1) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
-              dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
-            }
-          } else {
-            float4* d = reinterpret_cast<float4*>(
-                p.part + (static_cast<size_t>(kz) * p.M + m) * p.r_pad + j0 + c);
+          for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<float4*>(smem + lr_part_off(row, c / 4 + i, p.rc)) =
+                make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                            __uint_as_float(v[4 * i + 3]));
+        } else if (m < p.M) {
+          uint32_t hi[16], lo[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              if (empty_range)
-                d[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-              else
-                d[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            }
+          for (int i = 0; i < 16; ++i) {
+            const float a = __uint_as_float(v[2 * i]);
+            const float b = __uint_as_float(v[2 * i + 1]);
+            const uint16_t ha = to_bf16_bits(a), hb = to_bf16_bits(b);
+            hi[i] = static_cast<uint32_t>(ha) | (static_cast<uint32_t>(hb) << 16);
+            lo[i] = pack_bf16x2(a - bf16_bits_to_float(ha), b - bf16_bits_to_float(hb));
+          }
+          uint4* dh = reinterpret_cast<uint4*>(p.t_hi + static_cast<size_t>(m) * p.r_pad + j0 + c);
+          uint4* dl = reinterpret_cast<uint4*>(p.t_lo + static_cast<size_t>(m) * p.r_pad + j0 + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+            dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
           }
         }
       }
     }
   }
-  if (p.ksplit > 1) __threadfence();  // partials visible before this CTA counts itself in
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -235,58 +246,48 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
   }
   if (p.ksplit == 1) return;
 
-  // Split K: the last CTA of this tile to arrive sums the partials in
-  // split order and writes the bf16 pair, then re-arms the counter.  Every
-  // CTA counts itself in, also after a timeout, so the counter is back at
-  // zero when the grid ends.
-  __shared__ int s_last;
-  int* cnt = p.cnt + blockIdx.y * gridDim.x + blockIdx.x;
-  if (threadIdx.x == 0) s_last = atomicAdd(cnt, 1) == p.ksplit - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  // Split K: the CTAs of a cluster hold the partials of one tile; after the
+  // cluster barrier, CTA kz sums rows [kz * rpc, (kz + 1) * rpc) of every
+  // split's partial over distributed shared memory, in split order, and
+  // writes the bf16 pair.  Every CTA reaches both cluster barriers, also
+  // after a timeout.
+  cluster_sync();
   const int rows = min(128, p.M - m0);
+  const int rpc = (rows + p.ksplit - 1) / p.ksplit;
+  const int r0 = kz * rpc;
+  const int r1 = min(rows, r0 + rpc);
   const int q4 = wcols / 4;
-  const int total = rows * q4;
-  const size_t plane = static_cast<size_t>(p.M) * p.r_pad;
-  // Each thread sums kLrRedPer float4 columns at once, with every partial
-  // load issued before the first add (the sums are latency-bound).
-  constexpr int kLrRedPer = 4;
-  for (int i0 = threadIdx.x; i0 < total; i0 += kLrRedPer * blockDim.x) {
-    float4 v[kLrRedPer][kLrMaxSplit];
-    size_t off[kLrRedPer];
+  const int total = max(0, r1 - r0) * q4;
+  const uint32_t sbase = smem_u32(smem);
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int row = r0 + i / q4;
+    const int c4 = i % q4;
+    const uint32_t off = sbase + lr_part_off(row, c4, p.rc);
+    float4 v[kLrMaxSplit];
 #pragma unroll
-    for (int u = 0; u < kLrRedPer; ++u) {
-      const int i = i0 + u * blockDim.x;
-      off[u] = i < total ? static_cast<size_t>(m0 + i / q4) * p.r_pad + j0 + 4 * (i % q4) : 0;
+    for (int z = 0; z < kLrMaxSplit; ++z)
+      if (z < p.ksplit) v[z] = ld_shared_cluster_f4(mapa_shared(off, static_cast<uint32_t>(z)));
+    float4 acc = v[0];
 #pragma unroll
-      for (int z = 0; z < kLrMaxSplit; ++z)
-        if (i < total && z < p.ksplit) v[u][z] = __ldcg(reinterpret_cast<const float4*>(p.part + z * plane + off[u]));
-    }
-#pragma unroll
-    for (int u = 0; u < kLrRedPer; ++u) {
-      if (i0 + u * static_cast<int>(blockDim.x) >= total) break;
-      float4 acc = v[u][0];
-#pragma unroll
-      for (int z = 1; z < kLrMaxSplit; ++z)
-        if (z < p.ksplit) {
-          acc.x += v[u][z].x;
-          acc.y += v[u][z].y;
-          acc.z += v[u][z].z;
-          acc.w += v[u][z].w;
-        }
-      const uint16_t h0 = to_bf16_bits(acc.x), h1 = to_bf16_bits(acc.y);
-      const uint16_t h2 = to_bf16_bits(acc.z), h3 = to_bf16_bits(acc.w);
-      uint2 hv, lv;
-      hv.x = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-      hv.y = static_cast<uint32_t>(h2) | (static_cast<uint32_t>(h3) << 16);
-      lv.x = pack_bf16x2(acc.x - bf16_bits_to_float(h0), acc.y - bf16_bits_to_float(h1));
-      lv.y = pack_bf16x2(acc.z - bf16_bits_to_float(h2), acc.w - bf16_bits_to_float(h3));
-      *reinterpret_cast<uint2*>(p.t_hi + off[u]) = hv;
-      *reinterpret_cast<uint2*>(p.t_lo + off[u]) = lv;
-    }
+    for (int z = 1; z < kLrMaxSplit; ++z)
+      if (z < p.ksplit) {
+        acc.x += v[z].x;
+        acc.y += v[z].y;
+        acc.z += v[z].z;
+        acc.w += v[z].w;
+      }
+    const uint16_t h0 = to_bf16_bits(acc.x), h1 = to_bf16_bits(acc.y);
+    const uint16_t h2 = to_bf16_bits(acc.z), h3 = to_bf16_bits(acc.w);
+    uint2 hv, lv;
+    hv.x = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+    hv.y = static_cast<uint32_t>(h2) | (static_cast<uint32_t>(h3) << 16);
+    lv.x = pack_bf16x2(acc.x - bf16_bits_to_float(h0), acc.y - bf16_bits_to_float(h1));
+    lv.y = pack_bf16x2(acc.z - bf16_bits_to_float(h2), acc.w - bf16_bits_to_float(h3));
+    const size_t o = static_cast<size_t>(m0 + row) * p.r_pad + j0 + 4 * c4;
+    *reinterpret_cast<uint2*>(p.t_hi + o) = hv;
+    *reinterpret_cast<uint2*>(p.t_lo + o) = lv;
   }
-  if (threadIdx.x == 0) *cnt = 0;
+  cluster_sync();  // no CTA leaves while a peer still reads its partial
 }
 
 // =====================================================================
