@@ -71,8 +71,8 @@ constexpr int kTcEpiWarps = 8;   // two per lane quadrant, alternate 32-token bl
 constexpr int kTcXWarp = 2 + kTcConvWarps + kTcEpiWarps;  // x / low-rank producer
 constexpr int kTcThreads = 32 * (kTcXWarp + 1);
 constexpr int kTcMaxBT = 256;               // tokens per tile, at most
-constexpr int kTcSX = 4;                    // 32 KB slots: x chunks, A'/t chunks
-constexpr int kTcSQ = 4;                    // 16 KB slots: Q, two K steps each
+constexpr int kTcSX = 5;                    // 32 KB slots: x chunks, A'/t chunks
+constexpr int kTcSQ = 2;                    // 16 KB slots: Q, two K steps each
 constexpr int kTcNA = 4;                    // widened-Q stages in TMEM (two K steps, 64 columns each)
 constexpr int kTcXSlot = kTcMaxBT * kBK * 2;  // 32768
 constexpr int kTcQChunk = 128 * kBK;        // 8192: 128 rows x 64 codes
@@ -359,9 +359,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
     // Stages are numbered across this CTA's tiles (g); team t takes the
     // stages g = t (mod 2).  Within a team, warp (q, par) widens K step
     // 2s + par of the stage for the rows of lane quadrant q: one full
-    // 64-code row chunk per lane.  Stage g uses Q slot and TMEM stage
-    // g mod 4, in phase (g / 4) mod 2.
-    static_assert(kTcSQ == kTcNA, "Q slots and TMEM stages advance together");
+    // 64-code row chunk per lane.  Stage g uses Q slot g mod kTcSQ and
+    // TMEM stage g mod kTcNA, each in the phase of its own lap.
     const int cw = warp - 2;
     const int team = cw >> 3;
     const int q = warp & 3;
@@ -381,15 +380,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
       if (++ti == kTcTileRing) { ti = 0; tph ^= 1; }
       if (T < 0) break;
       for (long long g = gs + ((team - gs) & 1); g < gs + nS; g += 2) {
-        const int slot = static_cast<int>(g % kTcSQ);
-        const uint32_t ph = static_cast<uint32_t>((g / kTcSQ) & 1);
-        if (!__all_sync(0xffffffffu, mbar_wait(&q_full[slot], ph, p.watch, kErrTimeoutConvert))) { ok = false; break; }
+        const int qslot = static_cast<int>(g % kTcSQ);
+        const uint32_t qph = static_cast<uint32_t>((g / kTcSQ) & 1);
+        const int slot = static_cast<int>(g % kTcNA);  // TMEM stage
+        const uint32_t ph = static_cast<uint32_t>((g / kTcNA) & 1);
+        if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qslot], qph, p.watch, kErrTimeoutConvert))) { ok = false; break; }
         uint4 v[4];
-        const uint8_t* rb = sq + slot * kTcQSlot + par * kTcQChunk + row * 64;
+        const uint8_t* rb = sq + qslot * kTcQSlot + par * kTcQChunk + row * 64;
 #pragma unroll
         for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(rb + 16 * (j ^ sw));
         __syncwarp();
-        if (lane == 0) mbar_arrive(&q_empty[slot]);
+        if (lane == 0) mbar_arrive(&q_empty[qslot]);
         uint32_t w[32];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
