@@ -321,7 +321,7 @@ def run_crossover_suite(args):
     variants = {"stream": ll.LL_VARIANT_STREAM, "small": ll.LL_VARIANT_SMALL, "tc": ll.LL_VARIANT_TC,
                 "tc_pair": ll.LL_VARIANT_TC_PAIR, "auto": ll.LL_VARIANT_AUTO}
     points = []
-    for M in (1, 16, 32, 64, 96, 128, 192, 256, 384, 512, 1024, 2048, 4096):
+    for M in (1, 16, 32, 64, 96, 128, 192, 256, 384, 512, 1024, 2048, 4096, 8192, 16384):
         ll.ll_reserve(h, M)
         g = torch.Generator(device=dev)
         g.manual_seed(2000 + M)

@@ -64,11 +64,11 @@ enum {
   LL_ERR_SCRATCH_LIMIT = 8   /* request too large for ll_forward_noalloc's scratch */
 };
 
-/* Kernel variants for ll_set_variant.  AUTO: STREAM for M <= 64, SMALL
- * for 64 < M <= 128, TC above.  TC: one-CTA fused kernel, 128 features x
- * 256 tokens per tile, low-rank factor folded as A / scale (bf16 pair).
- * TC_PAIR: the same on CTA pairs (256 features per MMA); slower than TC on
- * every measured shape, kept selectable for comparison.  SMALL: one-CTA
+/* Kernel variants for ll_set_variant.  AUTO: STREAM for M <= 64, TC_PAIR
+ * for 64 < M <= 256, TC above (the measured crossovers).  TC: one-CTA fused
+ * kernel, 128 features x up to 256 tokens per tile, low-rank factor folded
+ * as A / scale (bf16 pair).  TC_PAIR: the same on CTA pairs (256 features
+ * per MMA, tiles as narrow as 32 tokens).  SMALL: one-CTA
  * kernel, 128 x 128 tiles, separate residual and low-rank accumulators.
  * STREAM (M <= 64 only; larger M runs SMALL): one CTA per 128 features
  * streaming Q in 32 KB boxes, all tokens in one MMA, exact A.  Every

@@ -233,6 +233,7 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st) {
 enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM };
 
 constexpr int kStreamMaxM = 64;
+constexpr int kPairMaxM = 256;
 
 Path choose_path(const ll_layer* h, int M) {
   if (h->variant == LL_VARIANT_TC) return PATH_TC1;
@@ -240,7 +241,10 @@ Path choose_path(const ll_layer* h, int M) {
   if (h->variant == LL_VARIANT_SMALL) return PATH_SMALL;
   if (h->variant == LL_VARIANT_STREAM) return M <= kStreamMaxM ? PATH_STREAM : PATH_SMALL;
   if (M <= kStreamMaxM) return PATH_STREAM;
-  return M > 128 ? PATH_TC1 : PATH_SMALL;
+  // Measured on the K = 4096, N = 16384 family: the CTA-pair kernel with
+  // its narrow tiles beats the 128 x 128 and one-CTA kernels up to 256
+  // tokens; above, the one-CTA kernel with its joint plan.
+  return M > kPairMaxM ? PATH_TC1 : PATH_TC2;
 }
 
 // CTAs of the streaming kernel: one per 128-feature tile, at most one per SM.
