@@ -125,6 +125,24 @@ int ll_reserve(ll_handle h, int max_M);
 /* Select a kernel variant (LL_VARIANT_AUTO picks by M). */
 int ll_set_variant(ll_handle h, int variant);
 
+/* The plan a forward of M tokens would follow on a layer of shape
+ * (N, K, r) with the given variant, on a GPU with num_sms SMs; host
+ * arithmetic only (no CUDA call, no handle), so it also runs without a GPU.
+ * The pages have no counterpart: this reports this library's dispatch
+ * (the kernel variants above) and its tile planning.
+ *   kernel:      the variant that runs (LL_VARIANT_TC, _TC_PAIR, _SMALL or
+ *                _STREAM; never AUTO).
+ *   tile_tokens: tokens per tile of that kernel (TC: the joint plan's
+ *                width; TC_PAIR: tokens per 256-feature pair tile; SMALL:
+ *                128; STREAM: M rounded up to 16).
+ *   lr_splits:   K splits of the down-projection t = x B^T (1 when r == 0).
+ * The CTA-pair plan assumes every pair of SMs can hold one cluster (a
+ * forward asks the occupancy calculator).  Any of the three out-pointers
+ * may be NULL.  Errors: LL_ERR_INVALID_ARG for shapes ll_create would
+ * reject, M < 1, num_sms < 2 or an unknown variant; LL_ERR_UNSUPPORTED for
+ * r > 512. */
+int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int *kernel, int *tile_tokens, int *lr_splits);
+
 /* Device status word of the handle: LL_OK, or LL_ERR_DEVICE_TIMEOUT if a
  * kernel of this handle gave up on a wait.  Synchronises the device;
  * call after the stream of the forward has been synchronised.  Reading

@@ -56,6 +56,8 @@ _SIGNATURES = {
     "ll_kernel_name": (ctypes.c_char_p, [_P, ctypes.c_int]),
     "ll_forward_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, _P]),
+    "ll_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               _P, _P, _P]),
 }
 
 
@@ -186,6 +188,18 @@ def ll_forward_noalloc(x, A, B, Q, scale, scale_mode: int, bias, y, M: int, N: i
                                  _addr(y), int(M), int(N), int(K), int(r), _stream(stream))
     if rc != LL_OK:
         raise LLError(rc, "ll_forward_noalloc")
+
+
+def ll_plan(N: int, K: int, r: int, M: int, num_sms: int, variant: int = 0):
+    """(kernel variant, tokens per tile, down-projection K splits) that a
+    forward of M tokens would use on an (N, K, r) layer with num_sms SMs.
+    Host arithmetic only; works without a GPU."""
+    k, bt, ks = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    rc = _lib.ll_plan(int(N), int(K), int(r), int(M), int(num_sms), int(variant), ctypes.byref(k), ctypes.byref(bt),
+                      ctypes.byref(ks))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_plan")
+    return k.value, bt.value, ks.value
 
 
 class LiteLinearLayer:

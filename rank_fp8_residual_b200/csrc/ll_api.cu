@@ -954,6 +954,47 @@ int ll_set_variant(ll_handle h, int variant) {
   return LL_OK;
 }
 
+int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int* kernel, int* tile_tokens, int* lr_splits) {
+  g_last_error = LL_OK;
+  if (N < 1 || K < 16 || r < 0 || (N % 8) != 0 || (K % 16) != 0 || M < 1 || num_sms < 2 ||
+      (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC && variant != LL_VARIANT_SMALL &&
+       variant != LL_VARIANT_TC_PAIR && variant != LL_VARIANT_STREAM))
+    return fail(LL_ERR_INVALID_ARG);
+  if (r > 512) return fail(LL_ERR_UNSUPPORTED);
+  // A handle-shaped view holding only what the planning reads.
+  ll_layer view;
+  view.N = N;
+  view.K = K;
+  view.r = r;
+  view.r_pad = (r + 31) / 32 * 32;
+  view.klr = (view.r_pad % 64 == 0) ? 64 : 32;
+  view.num_sms = num_sms;
+  view.variant = variant;
+  view.pair_clusters = num_sms / 2;
+  const Path path = choose_path(&view, M);
+  int kv = LL_VARIANT_SMALL, bt = 128;
+  switch (path) {
+    case PATH_TC1:
+      kv = LL_VARIANT_TC;
+      bt = M > 128 ? tc_tile_tokens(&view, M) : 256;
+      break;
+    case PATH_TC2:
+      kv = LL_VARIANT_TC_PAIR;
+      bt = tc2_tile_tokens(&view, M);
+      break;
+    case PATH_STREAM:
+      kv = LL_VARIANT_STREAM;
+      bt = (M + 15) / 16 * 16;
+      break;
+    case PATH_SMALL:
+      break;
+  }
+  if (kernel) *kernel = kv;
+  if (tile_tokens) *tile_tokens = bt;
+  if (lr_splits) *lr_splits = view.r_pad > 0 ? plan_lowrank(&view, M).ksplit : 1;
+  return LL_OK;
+}
+
 int ll_status(ll_handle h) {
   g_last_error = LL_OK;
   if (!h) return fail(LL_ERR_INVALID_ARG);

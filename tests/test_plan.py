@@ -1,0 +1,91 @@
+"""Host-side dispatch and tile planning (ll_plan): no GPU needed.
+
+The pins are the measured crossovers and plans recorded in the design
+notes: STREAM up to 64 tokens, CTA pairs up to 256, the one-CTA fused kernel
+above with 256-token tiles at the attention / FFN / sweep shapes.  The
+properties hold for every plan the library can make.
+"""
+import itertools
+
+import pytest
+
+import rank_fp8_residual_b200 as ll
+
+SMS = 148
+
+
+@pytest.mark.parametrize("N,K,r,M", [
+    (2048, 2048, 32, 3630),     # attention projection
+    (8192, 2048, 64, 3630),     # FFN up
+    (2048, 8192, 64, 3630),     # FFN down
+    (16384, 4096, 64, 8192),    # sweep point
+])
+def test_large_m_plans(N, K, r, M):
+    kernel, bt, ks = ll.ll_plan(N, K, r, M, SMS)
+    assert kernel == ll.LL_VARIANT_TC
+    assert bt == 256
+    assert ks == 1
+
+
+@pytest.mark.parametrize("M", [1, 16, 33, 64])
+def test_small_batch_streams(M):
+    kernel, bt, ks = ll.ll_plan(16384, 4096, 512, M, SMS)
+    assert kernel == ll.LL_VARIANT_STREAM
+    assert bt == (M + 15) // 16 * 16
+    assert 1 <= ks <= 8
+
+
+def test_auto_crossovers():
+    for M, want in [(64, ll.LL_VARIANT_STREAM), (65, ll.LL_VARIANT_TC_PAIR), (256, ll.LL_VARIANT_TC_PAIR),
+                    (257, ll.LL_VARIANT_TC), (4096, ll.LL_VARIANT_TC)]:
+        assert ll.ll_plan(16384, 4096, 64, M, SMS)[0] == want, M
+
+
+def test_forced_variants():
+    for M in (1, 100, 3000):
+        assert ll.ll_plan(4096, 4096, 64, M, SMS, ll.LL_VARIANT_TC)[0] == ll.LL_VARIANT_TC
+        assert ll.ll_plan(4096, 4096, 64, M, SMS, ll.LL_VARIANT_TC_PAIR)[0] == ll.LL_VARIANT_TC_PAIR
+        assert ll.ll_plan(4096, 4096, 64, M, SMS, ll.LL_VARIANT_SMALL)[0] == ll.LL_VARIANT_SMALL
+        want = ll.LL_VARIANT_STREAM if M <= 64 else ll.LL_VARIANT_SMALL
+        assert ll.ll_plan(4096, 4096, 64, M, SMS, ll.LL_VARIANT_STREAM)[0] == want
+
+
+def test_plan_properties():
+    Ns = (256, 2048, 16384)
+    Ks = (256, 4096, 8192)
+    rs = (0, 16, 32, 64, 200, 512)
+    Ms = (1, 63, 64, 65, 128, 129, 256, 257, 1000, 3630, 16384)
+    for N, K, r, M in itertools.product(Ns, Ks, rs, Ms):
+        kernel, bt, ks = ll.ll_plan(N, K, r, M, SMS)
+        assert kernel in (ll.LL_VARIANT_TC, ll.LL_VARIANT_TC_PAIR, ll.LL_VARIANT_STREAM)
+        if kernel == ll.LL_VARIANT_TC:
+            assert bt % 32 == 0 and 128 <= bt <= 256
+        elif kernel == ll.LL_VARIANT_TC_PAIR:
+            assert bt % 32 == 0 and 32 <= bt <= 256
+        else:
+            assert bt == (M + 15) // 16 * 16 and bt <= 64
+        n_kstep = (K + 63) // 64
+        if r == 0:
+            assert ks == 1
+        else:
+            assert 1 <= ks <= min(8, n_kstep)
+            if kernel == ll.LL_VARIANT_TC and M > 128 and ks > 1:
+                r_pad = (r + 31) // 32 * 32
+                rc = min(r_pad, 256)
+                ctas = (M + 127) // 128 * ((r_pad + rc - 1) // rc) * ks
+                assert ctas <= SMS
+
+
+def test_plan_rejects_bad_arguments():
+    with pytest.raises(ll.LLError):
+        ll.ll_plan(100, 4096, 64, 64, SMS)        # N % 8
+    with pytest.raises(ll.LLError):
+        ll.ll_plan(4096, 100, 64, 64, SMS)        # K % 16
+    with pytest.raises(ll.LLError):
+        ll.ll_plan(4096, 4096, 64, 0, SMS)        # M < 1
+    with pytest.raises(ll.LLError):
+        ll.ll_plan(4096, 4096, 64, 64, 1)         # num_sms < 2
+    with pytest.raises(ll.LLError):
+        ll.ll_plan(4096, 4096, 64, 64, SMS, 9)    # unknown variant
+    with pytest.raises(ll.LLError):
+        ll.ll_plan(4096, 4096, 513, 64, SMS)      # r > 512
