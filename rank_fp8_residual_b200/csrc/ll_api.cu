@@ -143,11 +143,13 @@ struct ll_layer {
   CUtensorMap tm_q3b2;  // the same view, 2 K chunks per box (fused single-CTA kernel)
   CUtensorMap c_xbt, c_thibt, c_tlobt;  // fused single-CTA kernel: x and t boxes of bt rows
   int c_bt = 0;
-  mutable int tcp_M = -1;  // M of the cached joint plan
+  mutable int tcp_M = -1;  // M of the cached joint plan (single-CTA kernel)
   mutable TcChoice tcp{};
+  mutable int tcp2_M = -1;  // M of the cached joint plan (CTA-pair kernel)
+  mutable TcChoice tcp2{};
   CUtensorMap c_x2p, c_thip, c_tlop;  // CTA-pair kernel: x and t boxes of bt2 / 2 rows
   int c_bt2 = 0;
-  int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
+  mutable int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
   int variant = LL_VARIANT_AUTO;
   int withhold = 0;
   uint64_t timeout_ns = 2000000000ull;
@@ -325,27 +327,51 @@ TcChoice plan_tc1(const ll_layer* h, int M) {
 
 int tc_tile_tokens(const ll_layer* h, int M) { return plan_tc1(h, M).bt; }
 
-int pair_cluster_count(ll_layer* h);
+int pair_cluster_count(const ll_layer* h);
 
-// Tokens per tile of the CTA-pair kernel (256 features per tile), by the
-// same model over the co-resident clusters; narrower tiles are allowed down
-// to 32 tokens for small M.
-int tc2_tile_tokens(ll_layer* h, int M) {
-  constexpr int kTileCost = 80;
+// The same joint plan for the CTA-pair kernel: tiles of 256 features over
+// the co-resident clusters, tile widths down to 32 tokens (small M), and a
+// down-projection CTA taking half a cluster's SMs.
+TcChoice plan_tc2(const ll_layer* h, int M) {
+  if (h->tcp2_M == M) return h->tcp2;
+  constexpr double kStageNsPerToken = 2.8;
+  constexpr double kTileFixedUs = 2.5;
+  constexpr double kLrFixedUs = 3.5;
+  constexpr double kLrCtaGBs = 70.0;
+  constexpr double kLrMaxGBs = 5500.0;
+  const int nK = (h->K + llk::kBK - 1) / llk::kBK;
+  const int nS = (nK + 1) / 2;
   const int n_fpairs = (h->N + 255) / 256;
   const int clusters = pair_cluster_count(h);
-  int best = 256;
-  long long best_cost = -1;
+  const int m_tiles = (M + 127) / 128;
+  const int rc = std::min(std::max(h->r_pad, 32), 256);
+  const int r_chunks = h->r_pad > 0 ? (h->r_pad + rc - 1) / rc : 0;
+  const double x_mb = 2.0 * M * h->K * r_chunks / 1e6;
+  TcChoice best{256, 1};
+  double best_t = -1;
   for (int bt = 256; bt >= 32; bt -= 32) {
     const long long tiles = static_cast<long long>(n_fpairs) * ((M + bt - 1) / bt);
-    const long long cost = (tiles + clusters - 1) / clusters * (bt + kTileCost);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = bt;
+    const double t_tile = kTileFixedUs + 0.3 * h->r_pad / 32 + nS * (bt + 32) * kStageNsPerToken * 1e-3;
+    const int ks_max = h->r_pad > 0 ? std::min(nK, llk::kLrMaxSplit) : 1;
+    for (int ks = 1; ks <= ks_max; ++ks) {
+      const int lr_ctas = h->r_pad > 0 ? m_tiles * r_chunks * ks : 0;
+      if (ks > 1 && lr_ctas > h->num_sms) break;
+      const int late = std::min((lr_ctas + 1) / 2, clusters);
+      const double t_lr =
+          h->r_pad > 0 ? kLrFixedUs + x_mb / std::min(std::max(lr_ctas, 1) * kLrCtaGBs, kLrMaxGBs) * 1e3 : 0.0;
+      const double t = tc_finish_us(tiles, clusters, late, t_tile, t_lr);
+      if (best_t < 0 || t < best_t * 0.99) {
+        best_t = t;
+        best = TcChoice{bt, ks};
+      }
     }
   }
+  h->tcp2_M = M;
+  h->tcp2 = best;
   return best;
 }
+
+int tc2_tile_tokens(ll_layer* h, int M) { return plan_tc2(h, M).bt; }
 
 struct LrPlan {
   int rc;            // column block of t per CTA (B box height)
@@ -374,16 +400,15 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   p.tmem_cols = next_pow2_ge32(p.rc);
   const int ctas = p.m_tiles * p.r_chunks;
   // The down-projection runs beside the fused kernels: as many splits as
-  // the joint plan gives next to the single-CTA kernel, three quarters of
-  // the SMs next to the CTA-pair kernel, and the SMs the streaming
-  // kernel's tiles leave free.  The other kernels wait for it, so it takes
-  // all SMs.
+  // the joint plans give next to the single-CTA and CTA-pair kernels, and
+  // the SMs the streaming kernel's tiles leave free.  The other kernels
+  // wait for it, so it takes all SMs.
   int budget = h->num_sms;
-  if (path == PATH_TC2) budget = std::max(1, h->num_sms * 3 / 4);
   if (path == PATH_STREAM) budget = std::max(1, h->num_sms - stream_ctas(h));
   int ks = std::max(1, budget / ctas);
   ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);
   if (path == PATH_TC1 && M > 128) ks = plan_tc1(h, M).ks;
+  if (path == PATH_TC2) ks = plan_tc2(h, M).ks;
   p.kb_per_split = (nK + ks - 1) / ks;
   p.ksplit = (nK + p.kb_per_split - 1) / p.kb_per_split;
   return p;
@@ -465,7 +490,7 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   return true;
 }
 
-int pair_cluster_count(ll_layer* h) {
+int pair_cluster_count(const ll_layer* h) {
   if (h->pair_clusters > 0) return h->pair_clusters;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(h->num_sms);
