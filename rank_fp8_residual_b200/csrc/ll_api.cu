@@ -448,7 +448,8 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
       ok &= make_map(&h->c_tlobt, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
     }
   }
-  if (choose_path(h, M) == PATH_TC2) {
+  {
+    // CTA-pair kernel maps (every M: any variant may be chosen later).
     const int bt2 = tc2_tile_tokens(h, M);
     const uint32_t hb = static_cast<uint32_t>(bt2 / 2);
     h->c_bt2 = bt2;
@@ -975,7 +976,6 @@ int ll_set_variant(ll_handle h, int variant) {
              variant != LL_VARIANT_TC_PAIR && variant != LL_VARIANT_STREAM))
     return fail(LL_ERR_INVALID_ARG);
   h->variant = variant;
-  h->c_M = -1;  // the per-call tensor maps depend on the kernel chosen
   return LL_OK;
 }
 
