@@ -11,12 +11,12 @@
 // Two CTAs of a cluster form one MMA of M = 256 output features: each CTA
 // widens its own 128 residual rows into its own TMEM stages (its half of
 // the A operand) and stages half of the token tile (its half of the B
-// operand) in its own shared memory.  So every SM writes 128 Q rows and
-// half of the x tile per K step into shared memory, and the pair MMA reads
-// each x half once for both tensor cores: about 44 KB of shared-memory
-// traffic per SM per K step against about 72 KB for the one-CTA kernel's
-// 128 x 256 tile, which is what bounds that kernel.  The accumulator of
-// each CTA holds its 128 features x up to 256 tokens.
+// operand) in its own shared memory.  So every SM stages 128 Q rows and
+// half of the x tile per K step, where the one-CTA kernel stages the whole
+// x tile; each tensor core still reads the whole B operand, half of it from
+// the peer.  Measured, a stage of eight MMAs takes about as long as in the
+// one-CTA kernel at N = 224 and 256.  The accumulator of each CTA holds its
+// 128 features x up to 256 tokens.
 //
 // The leader CTA (rank 0) issues the MMAs.  Its stage barrier a_full[s]
 // collects, for each stage of two K steps: its eight converter arrivals,
