@@ -285,8 +285,11 @@ double tc_finish_us(long long tiles, int sms, int late, double t_tile, double t_
   }
 }
 
-TcChoice plan_tc1(const ll_layer* h, int M) {
-  if (h->tcp_M == M) return h->tcp;
+// The finishing-time model over `slots` places for tiles of `feat`
+// features (SMs for the one-CTA kernel, clusters for the CTA pairs; one
+// down-projection CTA takes 1 / `sms_per_slot` of a place), tile widths
+// from 256 down to `bt_min` tokens.
+TcChoice plan_joint(const ll_layer* h, int M, int feat, int slots, int sms_per_slot, int bt_min) {
   constexpr double kStageNsPerToken = 2.8;  // per 2-K-step stage and (bt + 32) tokens
   constexpr double kTileFixedUs = 2.5;      // pipeline fill + epilogue per tile
   constexpr double kLrFixedUs = 3.5;        // down-projection launch, first loads, reduction
@@ -294,24 +297,24 @@ TcChoice plan_tc1(const ll_layer* h, int M) {
   constexpr double kLrMaxGBs = 5500.0;      // and of all of them together
   const int nK = (h->K + llk::kBK - 1) / llk::kBK;
   const int nS = (nK + 1) / 2;
-  const int n_ftiles = (h->N + 127) / 128;
+  const int n_ftiles = (h->N + feat - 1) / feat;
   const int m_tiles = (M + 127) / 128;
   const int rc = std::min(std::max(h->r_pad, 32), 256);
   const int r_chunks = h->r_pad > 0 ? (h->r_pad + rc - 1) / rc : 0;
   const double x_mb = 2.0 * M * h->K * r_chunks / 1e6;
   TcChoice best{256, 1};
   double best_t = -1;
-  for (int bt = 256; bt >= 128; bt -= 32) {
+  for (int bt = 256; bt >= bt_min; bt -= 32) {
     const long long tiles = static_cast<long long>(n_ftiles) * ((M + bt - 1) / bt);
     const double t_tile = kTileFixedUs + 0.3 * h->r_pad / 32 + nS * (bt + 32) * kStageNsPerToken * 1e-3;
     const int ks_max = h->r_pad > 0 ? std::min(nK, llk::kLrMaxSplit) : 1;
     for (int ks = 1; ks <= ks_max; ++ks) {
       const int lr_ctas = h->r_pad > 0 ? m_tiles * r_chunks * ks : 0;
       if (ks > 1 && lr_ctas > h->num_sms) break;
-      const int late = std::min(lr_ctas, h->num_sms);
+      const int late = std::min((lr_ctas + sms_per_slot - 1) / sms_per_slot, slots);
       const double t_lr =
-          h->r_pad > 0 ? kLrFixedUs + x_mb / std::min(late * kLrCtaGBs, kLrMaxGBs) * 1e3 : 0.0;
-      const double t = tc_finish_us(tiles, h->num_sms, late, t_tile, t_lr);
+          h->r_pad > 0 ? kLrFixedUs + x_mb / std::min(std::max(lr_ctas, 1) * kLrCtaGBs, kLrMaxGBs) * 1e3 : 0.0;
+      const double t = tc_finish_us(tiles, slots, late, t_tile, t_lr);
       // A wider tile or fewer down-projection CTAs unless the model gains
       // more than 1 %.
       if (best_t < 0 || t < best_t * 0.99) {
@@ -320,9 +323,15 @@ TcChoice plan_tc1(const ll_layer* h, int M) {
       }
     }
   }
-  h->tcp_M = M;
-  h->tcp = best;
   return best;
+}
+
+TcChoice plan_tc1(const ll_layer* h, int M) {
+  if (h->tcp_M != M) {
+    h->tcp = plan_joint(h, M, 128, h->num_sms, 1, 128);
+    h->tcp_M = M;
+  }
+  return h->tcp;
 }
 
 int tc_tile_tokens(const ll_layer* h, int M) { return plan_tc1(h, M).bt; }
@@ -333,42 +342,11 @@ int pair_cluster_count(const ll_layer* h);
 // the co-resident clusters, tile widths down to 32 tokens (small M), and a
 // down-projection CTA taking half a cluster's SMs.
 TcChoice plan_tc2(const ll_layer* h, int M) {
-  if (h->tcp2_M == M) return h->tcp2;
-  constexpr double kStageNsPerToken = 2.8;
-  constexpr double kTileFixedUs = 2.5;
-  constexpr double kLrFixedUs = 3.5;
-  constexpr double kLrCtaGBs = 70.0;
-  constexpr double kLrMaxGBs = 5500.0;
-  const int nK = (h->K + llk::kBK - 1) / llk::kBK;
-  const int nS = (nK + 1) / 2;
-  const int n_fpairs = (h->N + 255) / 256;
-  const int clusters = pair_cluster_count(h);
-  const int m_tiles = (M + 127) / 128;
-  const int rc = std::min(std::max(h->r_pad, 32), 256);
-  const int r_chunks = h->r_pad > 0 ? (h->r_pad + rc - 1) / rc : 0;
-  const double x_mb = 2.0 * M * h->K * r_chunks / 1e6;
-  TcChoice best{256, 1};
-  double best_t = -1;
-  for (int bt = 256; bt >= 32; bt -= 32) {
-    const long long tiles = static_cast<long long>(n_fpairs) * ((M + bt - 1) / bt);
-    const double t_tile = kTileFixedUs + 0.3 * h->r_pad / 32 + nS * (bt + 32) * kStageNsPerToken * 1e-3;
-    const int ks_max = h->r_pad > 0 ? std::min(nK, llk::kLrMaxSplit) : 1;
-    for (int ks = 1; ks <= ks_max; ++ks) {
-      const int lr_ctas = h->r_pad > 0 ? m_tiles * r_chunks * ks : 0;
-      if (ks > 1 && lr_ctas > h->num_sms) break;
-      const int late = std::min((lr_ctas + 1) / 2, clusters);
-      const double t_lr =
-          h->r_pad > 0 ? kLrFixedUs + x_mb / std::min(std::max(lr_ctas, 1) * kLrCtaGBs, kLrMaxGBs) * 1e3 : 0.0;
-      const double t = tc_finish_us(tiles, clusters, late, t_tile, t_lr);
-      if (best_t < 0 || t < best_t * 0.99) {
-        best_t = t;
-        best = TcChoice{bt, ks};
-      }
-    }
+  if (h->tcp2_M != M) {
+    h->tcp2 = plan_joint(h, M, 256, pair_cluster_count(h), 2, 32);
+    h->tcp2_M = M;
   }
-  h->tcp2_M = M;
-  h->tcp2 = best;
-  return best;
+  return h->tcp2;
 }
 
 int tc2_tile_tokens(ll_layer* h, int M) { return plan_tc2(h, M).bt; }
