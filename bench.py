@@ -54,7 +54,8 @@ def work_of(w, M=None):
     M = w.M if M is None else M
     K, N, r = w.K, w.N, w.r
     flops = 2.0 * M * (K * N + r * K + r * N)
-    bytes_ = 2.0 * M * K + N * K + 2.0 * N * r + 2.0 * r * K + 4.0 * N + 2.0 * N + 2.0 * M * N
+    scale_bytes = 4.0 * N if w.scale_mode == SCALE_PER_ROW else 4.0  # per-row [N] or per-tensor [1] fp32
+    bytes_ = 2.0 * M * K + N * K + 2.0 * N * r + 2.0 * r * K + scale_bytes + 2.0 * N + 2.0 * M * N
     # the fused kernel (x Q^T and the up-projection; B is read by the
     # down-projection kernel only)
     main_flops = 2.0 * M * N * (K + r)
