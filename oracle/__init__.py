@@ -18,6 +18,8 @@ import numpy as np
 
 EXACT = 0
 MIRROR = 1
+FP8ACT = 2     # x in x Q^T quantised per token to one e4m3fn term
+FP8SPLIT = 3   # x in x Q^T as the two-term e4m3fn expansion (diagnostic)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ll_oracle.c")
@@ -47,6 +49,13 @@ def lib():
         L.llo_enc_bf16_rne.restype = ctypes.c_uint16
         L.llo_enc_bf16_rne.argtypes = [ctypes.c_double]
         L.llo_num_threads.restype = ctypes.c_int
+        L.llo_enc_e4m3_rne.restype = ctypes.c_uint8
+        L.llo_enc_e4m3_rne.argtypes = [ctypes.c_double]
+        L.llo_token_exp.restype = ctypes.c_int
+        L.llo_token_exp.argtypes = [ctypes.c_double]
+        L.llo_quant_x.restype = ctypes.c_int
+        L.llo_quant_x.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         p = ctypes.c_void_p
         L.llo_forward.restype = ctypes.c_int
         L.llo_forward.argtypes = [ctypes.c_int] * 4 + [p, p, p, p, p, ctypes.c_int, p,
@@ -65,6 +74,29 @@ def dec_bf16(b: int) -> float:
 
 def enc_bf16_rne(v: float) -> int:
     return lib().llo_enc_bf16_rne(float(v))
+
+
+def enc_e4m3_rne(v: float) -> int:
+    return lib().llo_enc_e4m3_rne(float(v))
+
+
+def token_exp(amax: float) -> int:
+    return lib().llo_token_exp(float(amax))
+
+
+def quant_x(x, terms: int):
+    """Per-token e4m3fn quantisation of x (uint16 bf16 bits [M, K]):
+    returns (e [M] int32, hi [M, K] uint8, lo [M, K] uint8 or None), with
+    x[m, k] ~= 2^e[m] * (hi + lo) (lo only for terms == 2)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    M, K = x.shape
+    e = np.zeros(M, dtype=np.int32)
+    hi = np.zeros((M, K), dtype=np.uint8)
+    lo = np.zeros((M, K), dtype=np.uint8) if terms == 2 else None
+    rc = lib().llo_quant_x(M, K, _ptr(x), int(terms), _ptr(e), _ptr(hi), _ptr(lo))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return e, hi, lo
 
 
 def num_threads() -> int:

@@ -31,6 +31,20 @@
  *                   fused kernel cast-for-cast; modegpt page,
  *                   MoDeGPTLowRankLinear.forward applies F.linear(x, V) in
  *                   the activation dtype).  Diagnostic only.
+ *   LLO_FP8ACT (2): the FP8-activation reading.  The residual product
+ *                   x Q^T uses x quantised per token to e4m3fn,
+ *                   x ~= 2^e_m * q_m, where 2^e_m is the smallest power of
+ *                   two with max_k |x[m][k]| <= 448 * 2^e_m and q_m is the
+ *                   round-to-nearest-even e4m3fn code of x / 2^e_m (README
+ *                   "Features": e4m3fn is the FP8 format of the layer; its
+ *                   benchmark's fused "Accel" kernel; the per-token power of
+ *                   two is the plainest scale that keeps every product
+ *                   exact).  t = x B^T keeps the unquantised x.
+ *   LLO_FP8SPLIT (3): x in the residual product is the two-term e4m3fn
+ *                   expansion 2^e_m * (hi + lo), hi as in LLO_FP8ACT and
+ *                   lo the e4m3fn rounding of x / 2^e_m - hi.  Diagnostic
+ *                   mirror of the two-term kernel (graded against
+ *                   LLO_EXACT).
  *
  * Parity status: every function here is pinned by the tests under
  * tests/test_oracle_*.py (exhaustive decoder checks against torch's
@@ -47,6 +61,8 @@
 
 #define LLO_EXACT 0
 #define LLO_MIRROR 1
+#define LLO_FP8ACT 2
+#define LLO_FP8SPLIT 3
 #define LLO_SCALE_PER_TENSOR 0
 #define LLO_SCALE_PER_ROW 1
 
@@ -118,6 +134,95 @@ uint16_t llo_enc_bf16_rne(double v)
     return sign | (uint16_t)((u >> 16) & 0x7FFFu);
 }
 
+/* Round a binary64 value to e4m3fn, nearest with ties to the even code,
+ * and return the code.  Magnitudes above 448 give 448 (the largest finite
+ * code; e4m3fn has no infinity), NaN gives 0x7F.  Written as a search
+ * over the 127 finite non-negative codes, whose values are given in
+ * `pos` (pos[c] = llo_dec_e4m3(c), c = 0x00 .. 0x7E): the nearest value
+ * wins, and of two equally near ones (always adjacent codes) the even
+ * code. */
+static uint8_t enc_e4m3_search(double v, const double *pos)
+{
+    if (isnan(v))
+        return 0x7Fu;
+    uint8_t sign = signbit(v) ? 0x80u : 0u;
+    double a = fabs(v);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(pos[c] - a);
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+static void e4m3_positive_values(double *pos)
+{
+    for (int c = 0; c <= 0x7E; ++c)
+        pos[c] = llo_dec_e4m3((uint8_t)c);
+}
+
+uint8_t llo_enc_e4m3_rne(double v)
+{
+    double pos[0x7F];
+    e4m3_positive_values(pos);
+    return enc_e4m3_search(v, pos);
+}
+
+/* Per-token exponent of the FP8-activation readings: the smallest integer
+ * e with amax <= 448 * 2^e, limited to [-126, 126] (so that 2^e and 2^-e
+ * are normal binary32 numbers); 0 for amax == 0. */
+int llo_token_exp(double amax)
+{
+    if (!(amax > 0.0))
+        return 0;
+    int e = -126;
+    while (e < 126 && amax > ldexp(448.0, e))
+        ++e;
+    return e;
+}
+
+/* Quantise one token row: returns e_m and writes the codes hi[k] (and
+ * lo[k] when terms == 2) of u = x[k] / 2^e_m:  hi = e4m3(u),
+ * lo = e4m3(u - hi).  `pos` as for enc_e4m3_search. */
+static int quant_row(const uint16_t *xr, int K, int terms, const double *pos, uint8_t *hi, uint8_t *lo)
+{
+    double amax = 0.0;
+    for (int k = 0; k < K; ++k) {
+        double a = fabs(llo_dec_bf16(xr[k]));
+        if (a > amax)
+            amax = a;
+    }
+    int e = llo_token_exp(amax);
+    for (int k = 0; k < K; ++k) {
+        double u = ldexp(llo_dec_bf16(xr[k]), -e);
+        uint8_t h = enc_e4m3_search(u, pos);
+        hi[k] = h;
+        if (terms == 2)
+            lo[k] = enc_e4m3_search(u - llo_dec_e4m3(h), pos);
+    }
+    return e;
+}
+
+/* The per-token quantisation of x [M][K] used by the FP8-activation
+ * readings: e_out [M], hi [M][K] and, for terms == 2, lo [M][K].
+ * Returns 0, or -1 on bad arguments. */
+int llo_quant_x(int M, int K, const uint16_t *x, int terms, int *e_out, uint8_t *hi, uint8_t *lo)
+{
+    if (M < 0 || K < 0 || (terms != 1 && terms != 2) || (M > 0 && (!x || !e_out || !hi)) ||
+        (M > 0 && terms == 2 && !lo))
+        return -1;
+    double pos[0x7F];
+    e4m3_positive_values(pos);
+    for (int m = 0; m < M; ++m)
+        e_out[m] = quant_row(x + (size_t)m * (size_t)K, K, terms, pos, hi + (size_t)m * (size_t)K,
+                             terms == 2 ? lo + (size_t)m * (size_t)K : NULL);
+    return 0;
+}
+
 /*
  * The forward pass for the rows listed in `rows` (or all M rows when
  * rows == NULL), written out as the definition:
@@ -126,6 +231,8 @@ uint16_t llo_enc_bf16_rne(double v)
  *   yq[n]   = sum_k x[m][k] * Q[n][k]                      (decoded e4m3)
  *   ylr[n]  = sum_j t[j] * A[n][j]
  *   y[i][n] = s_n * yq[n] + ylr[n] + bias[n]
+ *
+ * In the FP8 modes yq uses the quantised row (see the mode list above).
  *
  * s_n = scale[n] (per row) or scale[0] (per tensor); bias may be NULL.
  * Output y is [nrows][N] binary64, where nrows = M when rows == NULL.
@@ -139,7 +246,7 @@ int llo_forward(int M, int K, int N, int r,
 {
     if (M < 0 || K < 0 || N < 0 || r < 0 || !y)
         return -1;
-    if (mode != LLO_EXACT && mode != LLO_MIRROR)
+    if (mode != LLO_EXACT && mode != LLO_MIRROR && mode != LLO_FP8ACT && mode != LLO_FP8SPLIT)
         return -1;
     if (scale_mode != LLO_SCALE_PER_TENSOR && scale_mode != LLO_SCALE_PER_ROW)
         return -1;
@@ -159,6 +266,8 @@ int llo_forward(int M, int K, int N, int r,
     double dq[256];
     for (int c = 0; c < 256; ++c)
         dq[c] = llo_dec_e4m3((uint8_t)c);
+    double pos[0x7F];
+    e4m3_positive_values(pos);
     double *Bd = NULL, *Ad = NULL;
     if (r > 0) {
         Bd = (double *)malloc(sizeof(double) * (size_t)r * (size_t)(K > 0 ? K : 1));
@@ -178,8 +287,11 @@ int llo_forward(int M, int K, int N, int r,
 #pragma omp parallel
     {
         double *xd = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+        double *xq = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+        uint8_t *qh = (uint8_t *)malloc((size_t)(K > 0 ? K : 1));
+        uint8_t *ql = (uint8_t *)malloc((size_t)(K > 0 ? K : 1));
         double *t = (double *)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1));
-        if (!xd || !t) {
+        if (!xd || !xq || !qh || !ql || !t) {
 #pragma omp atomic write
             fail = 1;
         } else {
@@ -189,6 +301,19 @@ int llo_forward(int M, int K, int N, int r,
                 const uint16_t *xr = x + (size_t)m * (size_t)K;
                 for (int k = 0; k < K; ++k)
                     xd[k] = llo_dec_bf16(xr[k]);
+                /* the row that enters x Q^T */
+                const double *xr_q = xd;
+                if (mode == LLO_FP8ACT || mode == LLO_FP8SPLIT) {
+                    int terms = mode == LLO_FP8ACT ? 1 : 2;
+                    int e = quant_row(xr, K, terms, pos, qh, ql);
+                    for (int k = 0; k < K; ++k) {
+                        double v = llo_dec_e4m3(qh[k]);
+                        if (terms == 2)
+                            v += llo_dec_e4m3(ql[k]);
+                        xq[k] = ldexp(v, e);
+                    }
+                    xr_q = xq;
+                }
                 /* t = x B^T */
                 for (int j = 0; j < r; ++j) {
                     const double *bj = Bd + (size_t)j * (size_t)K;
@@ -202,7 +327,7 @@ int llo_forward(int M, int K, int N, int r,
                     const uint8_t *qn = Q + (size_t)n * (size_t)K;
                     double yq = 0.0;
                     for (int k = 0; k < K; ++k)
-                        yq += xd[k] * dq[qn[k]];
+                        yq += xr_q[k] * dq[qn[k]];
                     double ylr = 0.0;
                     const double *an = Ad ? Ad + (size_t)n * (size_t)r : NULL;
                     for (int j = 0; j < r; ++j)
@@ -214,6 +339,9 @@ int llo_forward(int M, int K, int N, int r,
             }
         }
         free(xd);
+        free(xq);
+        free(qh);
+        free(ql);
         free(t);
     }
     free(Bd);
