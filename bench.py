@@ -81,6 +81,8 @@ KERNEL_SOURCES = {
     "ll_main_kernel": ["ll_kernels.cuh", "ptx.cuh"],
     "ll_lrdown_kernel": ["ll_kernels.cuh", "ptx.cuh"],
     "ll_stream_kernel": ["ll_stream.cuh", "ll_kernels.cuh", "ptx.cuh"],
+    "ll_f8_kernel": ["ll_f8.cuh", "ll_kernels.cuh", "ptx.cuh"],
+    "ll_xsplit_kernel": ["ll_f8.cuh", "ll_kernels.cuh", "ptx.cuh"],
 }
 
 
@@ -374,7 +376,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="auto", choices=["auto", "tc", "tc_pair", "small", "stream"],
+    ap.add_argument("--variant", default="auto",
+                    choices=["auto", "tc", "tc_pair", "small", "stream", "fp8_split", "fp8_act"],
                     help="kernel variant (auto picks by token count)")
     ap.add_argument("--suite", default=None, choices=["page", "crossover"],
                     help="page: the README's LTX-Video FFN shapes, count-weighted total; "
@@ -413,7 +416,8 @@ def main():
                       inp.bias.to(dev) if inp.bias is not None else None)
     h = layer.handle
     ll.ll_set_variant(h, {"auto": ll.LL_VARIANT_AUTO, "tc": ll.LL_VARIANT_TC, "tc_pair": ll.LL_VARIANT_TC_PAIR,
-                          "small": ll.LL_VARIANT_SMALL, "stream": ll.LL_VARIANT_STREAM}[args.variant])
+                          "small": ll.LL_VARIANT_SMALL, "stream": ll.LL_VARIANT_STREAM,
+                          "fp8_split": ll.LL_VARIANT_FP8_SPLIT, "fp8_act": ll.LL_VARIANT_FP8_ACT}[args.variant])
     ll.ll_reserve(h, w.M)
     x = inp.x.to(dev)
     y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)

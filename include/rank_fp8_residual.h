@@ -64,37 +64,59 @@ enum {
   LL_ERR_SCRATCH_LIMIT = 8   /* request too large for ll_forward_noalloc's scratch */
 };
 
-/* Kernel variants for ll_set_variant.  AUTO: STREAM for M <= 64, TC_PAIR
- * for 64 < M <= 256, TC above (the measured crossovers).  TC: one-CTA fused
+/* Kernel variants for ll_set_variant (no counterpart on the pages).  AUTO:
+ * STREAM for M <= 64, TC_PAIR for 64 < M <= 256, TC above (the measured
+ * crossovers).  TC: one-CTA fused
  * kernel, 128 features x up to 256 tokens per tile, low-rank factor folded
  * as A / scale (bf16 pair).  TC_PAIR: the same on CTA pairs (256 features
  * per MMA, tiles as narrow as 32 tokens).  SMALL: one-CTA
  * kernel, 128 x 128 tiles, separate residual and low-rank accumulators.
  * STREAM (M <= 64 only; larger M runs SMALL): one CTA per 128 features
- * streaming Q in 32 KB boxes, all tokens in one MMA, exact A.  Every
- * variant meets the same accuracy bound. */
+ * streaming Q in 32 KB boxes, all tokens in one MMA, exact A.  FP8_SPLIT:
+ * CTA pairs on e4m3 tensor cores (kind::f8f6f4) with Q as stored and x
+ * carried per token as the two-term e4m3fn expansion of ll_quantize_x.
+ * These variants meet the same accuracy bound.  FP8_ACT: the same kernel
+ * on one e4m3fn term per token, the FP8-activation variant: its result is
+ * the layer's formula evaluated on x quantised per token as by
+ * ll_quantize_x with terms == 1 (that rounding of x is part of the
+ * variant's definition). */
 enum {
   LL_VARIANT_AUTO = 0,
   LL_VARIANT_TC = 1,
   LL_VARIANT_SMALL = 2,
   LL_VARIANT_TC_PAIR = 3,
-  LL_VARIANT_STREAM = 4
+  LL_VARIANT_STREAM = 4,
+  LL_VARIANT_FP8_SPLIT = 5,
+  LL_VARIANT_FP8_ACT = 6
 };
 
-/* Create a layer with N output features, K input features and rank r on
+/* LiteLinear README, "Usage": the layer constructor
+ * LiteLinear(in_features, out_features, bias, rank) -- here K = in_features,
+ * N = out_features, r = rank, and whether a bias exists is decided by
+ * ll_set_weights.  The scale granularity (one per output feature or one
+ * per tensor) is not stated on the page; scale_mode selects it.
+ *
+ * Create a layer with N output features, K input features and rank r on
  * the current CUDA device.  Requires N >= 1 and N % 8 == 0, K >= 16 and
  * K % 16 == 0, 0 <= r <= 512, scale_mode one of LL_SCALE_*.  The handle is
  * host-allocated; device memory for the factors is allocated here.
- * Returns NULL on error (see ll_last_error()). */
+ * Returns NULL on error (see ll_last_error()): LL_ERR_INVALID_ARG for bad
+ * sizes or mode, LL_ERR_UNSUPPORTED for r > 512 or a GPU other than
+ * sm_100, LL_ERR_OOM / LL_ERR_CUDA when the device allocation fails. */
 ll_handle ll_create(int N, int K, int r, int scale_mode);
 
-/* Copy the factors into handle-owned device memory (device-to-device;
+/* LiteLinear README, "Features": the factors a converted layer holds, its
+ * state-dict keys A, B, Q_fp8, Q_scale_inv and bias (A, B bf16; Q_fp8
+ * e4m3fn; Q_scale_inv is the "scale" of the introduction's formula and is
+ * applied as a multiplier).
+ *
+ * Copy the factors into handle-owned device memory (device-to-device;
  * the caller may free its buffers once the call returns -- the call
  * synchronises the device).  A: bf16 [N, r]; B: bf16 [r, K] (both may be
  * NULL when r == 0); Q: e4m3fn codes [N, K]; scale: fp32 [N] or [1] by
- * the layer's scale_mode; bias: bf16 [N] or NULL.  All non-NULL pointers
- * must be 16-byte aligned device pointers except scale and bias (4- and
- * 2-byte aligned).  The rank is zero-padded internally to a multiple of
+ * the layer's scale_mode; bias: bf16 [N] or NULL.  A, B and Q must be
+ * 16-byte aligned device pointers, scale 4-byte and bias 2-byte aligned
+ * (LL_ERR_INVALID_ARG otherwise).  The rank is zero-padded internally to a multiple of
  * 32 (exact).  The call also prepares A / scale as a bf16 pair for the
  * fused large-M kernel.  Returns LL_ERR_NAN_CODE if any Q code is 0x7F or
  * 0xFF; LL_ERR_INVALID_ARG for null/misaligned/non-device pointers or a
@@ -103,7 +125,10 @@ ll_handle ll_create(int N, int K, int r, int scale_mode);
 int ll_set_weights(ll_handle h, const void *A, const void *B, const void *Q, const float *scale,
                    const void *bias);
 
-/* y = forward(x) for M rows on `stream` (a cudaStream_t; NULL is the
+/* LiteLinear README, "Usage": y = layer(x), evaluating the introduction's
+ * display formula y = (x B^T) A^T + scale * (x Q_fp8^T) + bias.
+ *
+ * y = forward(x) for M rows on `stream` (a cudaStream_t; NULL is the
  * legacy default stream).  x: bf16 [M, K], y: bf16 [M, N], both 16-byte
  * aligned device pointers that must not overlap.  M == 0 is a no-op.  The
  * call is asynchronous; x and y are borrowed until the stream reaches the
@@ -112,17 +137,21 @@ int ll_set_weights(ll_handle h, const void *A, const void *B, const void *Q, con
  * beforehand to avoid that, e.g. before graph capture). */
 int ll_forward(ll_handle h, const void *x, void *y, int M, void *stream);
 
-/* ll_forward on HOST buffers: copies x (host, bf16 [M, K]) to the device,
+/* No counterpart on the pages: the forward from host memory.
+ *
+ * ll_forward on HOST buffers: copies x (host, bf16 [M, K]) to the device,
  * runs the forward and copies y back to the host (bf16 [M, N]), all on
  * `stream`.  Pinned host buffers make the copies asynchronous; the caller
  * synchronises the stream before reading y.  Device staging buffers are
  * handle-owned and grown on demand. */
 int ll_forward_host(ll_handle h, const void *x_host, void *y_host, int M, void *stream);
 
-/* Pre-size the workspace for forwards of up to max_M rows (synchronous). */
+/* No counterpart on the pages.  Pre-size the workspace for forwards of up
+ * to max_M rows (synchronous). */
 int ll_reserve(ll_handle h, int max_M);
 
-/* Select a kernel variant (LL_VARIANT_AUTO picks by M). */
+/* No counterpart on the pages.  Select a kernel variant (LL_VARIANT_AUTO
+ * picks by M).  LL_ERR_INVALID_ARG for an unknown variant. */
 int ll_set_variant(ll_handle h, int variant);
 
 /* The plan a forward of M tokens would follow on a layer of shape
@@ -143,42 +172,61 @@ int ll_set_variant(ll_handle h, int variant);
  * r > 512. */
 int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int *kernel, int *tile_tokens, int *lr_splits);
 
-/* Device status word of the handle: LL_OK, or LL_ERR_DEVICE_TIMEOUT if a
+/* No counterpart on the pages.  Device status word of the handle: LL_OK, or LL_ERR_DEVICE_TIMEOUT if a
  * kernel of this handle gave up on a wait.  Synchronises the device;
  * call after the stream of the forward has been synchronised.  Reading
  * the status clears it. */
 int ll_status(ll_handle h);
 
-/* Debug controls: timeout_ns bounds every device-side wait (default 2 s);
+/* No counterpart on the pages.  Debug controls: timeout_ns bounds every device-side wait (default 2 s);
  * withhold_producer != 0 makes the main kernel's loader issue nothing, so
  * its consumers run into the timeout (used to test the timeout path). */
 int ll_set_debug(ll_handle h, int withhold_producer, uint64_t timeout_ns);
 
-/* Release the handle and all device memory it owns (synchronises). */
+/* The per-token e4m3fn quantisation of activations that the FP8-operand
+ * variants apply before the residual product (the FP8-activation reading
+ * of the README's "Features" list and its fused benchmark kernel): for
+ * each token row m of x (bf16 [M, K], device, 16-byte aligned) it writes
+ * e_out[m] (int32 [M]), the smallest e in [-126, 126] with
+ * max_k |x[m, k]| <= 448 * 2^e (0 for an all-zero row), and the e4m3fn
+ * codes hi[m, k] = rne(x[m, k] / 2^e) (uint8 [M, K], 16-byte aligned);
+ * with terms == 2 also lo[m, k] = rne(x[m, k] / 2^e - hi[m, k]), so that
+ * 2^e * (hi + lo) equals x wherever |x| >= 2^e / 4 and lies within
+ * 2^(e - 10) of it elsewhere.  rne rounds to the nearest e4m3fn value,
+ * ties to the even code.  K % 16 == 0.  Asynchronous on `stream`;
+ * LL_ERR_INVALID_ARG for bad sizes, terms, or null / misaligned /
+ * non-device pointers. */
+int ll_quantize_x(const void *x, int M, int K, int terms, int *e_out, void *hi, void *lo, void *stream);
+
+/* No counterpart on the pages.  Release the handle and all device memory
+ * it owns (synchronises). */
 void ll_destroy(ll_handle h);
 
-/* Code of the last failed call on this host thread (LL_OK if none). */
+/* No counterpart on the pages.  Code of the last failed call on this host
+ * thread (LL_OK if none). */
 int ll_last_error(void);
 
-/* Static description of a status code. */
+/* No counterpart on the pages.  Static description of a status code. */
 const char *ll_status_string(int code);
 
-/* Number of kernels the last ll_forward on this handle launched. */
+/* No counterpart on the pages.  Number of kernels the last ll_forward on
+ * this handle launched. */
 int ll_last_launch_count(ll_handle h);
 
-/* Profiling mode (enable != 0): every later ll_forward records CUDA events
+/* No counterpart on the pages.  Profiling mode (enable != 0): every later ll_forward records CUDA events
  * on its stream around each kernel it launches, and launches them without
  * programmatic overlap so each duration is that kernel's alone.  All work
  * is still done.  Off by default. */
 int ll_set_profiling(ll_handle h, int enable);
 
-/* Device durations in milliseconds of the kernels the last profiled
+/* No counterpart on the pages.  Device durations in milliseconds of the kernels the last profiled
  * ll_forward launched, in launch order, written to ms[0 .. n).  Waits for
  * the events.  Returns the number of kernels (may exceed n), or -1 if the
  * last forward was not profiled. */
 int ll_kernel_times(ll_handle h, float *ms, int n);
 
-/* Name of the i-th kernel of the last ll_forward (static string), or NULL. */
+/* No counterpart on the pages.  Name of the i-th kernel of the last
+ * ll_forward (static string), or NULL. */
 const char *ll_kernel_name(ll_handle h, int i);
 
 /* ---------------------------------------------------------------------
@@ -206,7 +254,7 @@ const char *ll_kernel_name(ll_handle h, int i);
  * when r == 0), Q e4m3fn codes [N, K], scale fp32 [N] (LL_SCALE_PER_ROW) or
  * [1] (LL_SCALE_PER_TENSOR), bias bf16 [N] or NULL, y bf16 [M, N]; all
  * device pointers of the current device; x, y, A, B and Q 16-byte
- * aligned, scale 4-byte, bias 2-byte; y must not overlap x.  Shapes follow
+ * aligned, scale 4-byte, bias 2-byte; y must not overlap any input.  Shapes follow
  * ll_create (N % 8 == 0, K % 16 == 0, K >= 16, 0 <= r <= 512) and, since
  * A is read in place, r % 8 == 0.  M == 0 is a no-op.
  *
@@ -227,12 +275,16 @@ const char *ll_kernel_name(ll_handle h, int i);
  * threads) race on the array and give wrong results: order them on one
  * stream or with events.
  *
- * Set-up: the first call on each device (made with that device current)
- * looks up the array's device address and sets kernel attributes; make
- * that first call before any stream capture.
+ * Set-up: the first successful call on each device (made with that
+ * device current) looks up the array's device address and sets kernel
+ * attributes; make that first call before any stream capture.  A set-up
+ * that fails is not kept: the next call tries again.  cudaDeviceReset
+ * invalidates the set-up; do not call this entry point on a device after
+ * resetting it in the same process.
  *
- * Errors: LL_ERR_INVALID_ARG for bad shapes, modes, null / misaligned /
- * non-device pointers or overlap; LL_ERR_UNSUPPORTED for r % 8 != 0;
+ * Errors: LL_ERR_INVALID_ARG for bad shapes, modes, null / misaligned
+ * pointers, pointers that are not device memory of the current device, or
+ * y overlapping any input; LL_ERR_UNSUPPORTED for r % 8 != 0;
  * LL_ERR_SCRATCH_LIMIT as above; LL_ERR_CUDA when a launch fails.  A
  * device-side wait that runs past its limit (2 s) ends the kernels early
  * and leaves y incomplete; this call has no way to report that

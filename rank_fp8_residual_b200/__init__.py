@@ -35,6 +35,8 @@ LL_VARIANT_TC = 1
 LL_VARIANT_SMALL = 2
 LL_VARIANT_TC_PAIR = 3
 LL_VARIANT_STREAM = 4
+LL_VARIANT_FP8_SPLIT = 5
+LL_VARIANT_FP8_ACT = 6
 
 # Every symbol the header declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -56,6 +58,7 @@ _SIGNATURES = {
     "ll_kernel_name": (ctypes.c_char_p, [_P, ctypes.c_int]),
     "ll_forward_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, _P]),
+    "ll_quantize_x": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P]),
     "ll_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                _P, _P, _P]),
 }
@@ -188,6 +191,15 @@ def ll_forward_noalloc(x, A, B, Q, scale, scale_mode: int, bias, y, M: int, N: i
                                  _addr(y), int(M), int(N), int(K), int(r), _stream(stream))
     if rc != LL_OK:
         raise LLError(rc, "ll_forward_noalloc")
+
+
+def ll_quantize_x(x, M: int, K: int, terms: int, e_out, hi, lo=None, stream=None) -> None:
+    """Per-token e4m3fn codes of x (bf16 [M, K]): e_out int32 [M], hi uint8
+    [M, K] and, for terms == 2, lo uint8 [M, K] (device buffers)."""
+    rc = _lib.ll_quantize_x(_addr(x), int(M), int(K), int(terms), _addr(e_out), _addr(hi), _addr(lo),
+                            _stream(stream))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_quantize_x")
 
 
 def ll_plan(N: int, K: int, r: int, M: int, num_sms: int, variant: int = 0):

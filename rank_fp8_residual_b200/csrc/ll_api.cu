@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -18,6 +19,7 @@
 #include "ll_tc.cuh"
 #include "ll_tc2.cuh"
 #include "ll_stream.cuh"
+#include "ll_f8.cuh"
 
 namespace {
 
@@ -90,6 +92,23 @@ bool is_device_ptr(const void* p) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Device memory (or managed memory) of device `dev`.
+bool is_device_ptr_on(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+}
+
+// Byte ranges [a, a + na) and [b, b + nb) intersect.
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const char* pa = static_cast<const char*>(a);
+  const char* pb = static_cast<const char*>(b);
+  return na > 0 && nb > 0 && pa < pb + nb && pb < pa + na;
+}
+
 int next_pow2_ge32(int v) {
   int p = 32;
   while (p < v) p <<= 1;
@@ -126,6 +145,18 @@ struct ll_layer {
   int ws_M = 0;
   uint16_t* t_hi = nullptr;
   uint16_t* t_lo = nullptr;
+  // FP8-operand path: per-token exponents and e4m3 codes of x
+  int ws8_M = 0;
+  int* e_tok = nullptr;
+  uint8_t* xh = nullptr;
+  uint8_t* xl = nullptr;
+  int* f8_cnt = nullptr;     // arrival counters of K-split tiles, [tiles of ws8_M rows][2][4]
+  size_t f8_cnt_n = 0;
+  float* f8_part = nullptr;  // fp32 partial tiles, two slots per CTA pair
+  CUtensorMap tm_q128, tm_ahi32, tm_alo32;     // set-time maps of the FP8-operand kernel
+  CUtensorMap c_xh, c_xl, c_thi32, c_tlo32, c_y64;  // per-call maps of the FP8-operand kernel
+  bool c_f8 = false;                           // the per-call FP8 maps are built
+  mutable int f8_clusters = 0;                 // co-resident clusters of the FP8-operand kernel
   // host-buffer forward staging
   void* dx = nullptr;
   void* dy = nullptr;
@@ -182,6 +213,11 @@ void free_layer_mem(ll_layer* h) {
   cudaFree(h->t_lo);
   cudaFree(h->dx);
   cudaFree(h->dy);
+  cudaFree(h->e_tok);
+  cudaFree(h->xh);
+  cudaFree(h->xl);
+  cudaFree(h->f8_cnt);
+  cudaFree(h->f8_part);
 }
 
 int set_smem_attrs_once() {
@@ -203,6 +239,9 @@ int set_smem_attrs_once() {
       rc = 1;
     if (cudaFuncSetAttribute(llk::ll_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::st_smem_max()) != cudaSuccess)
+      rc = 1;
+    if (cudaFuncSetAttribute(llk::ll_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             llk::f8_smem_bytes()) != cudaSuccess)
       rc = 1;
   });
   return rc;
@@ -232,12 +271,60 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st) {
   return LL_OK;
 }
 
-enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM };
+// Grow the FP8-operand path's buffers (token exponents, e4m3 codes of x)
+// to `M` rows (stream-ordered).
+int f8_cluster_count(const ll_layer* h);
+
+int ensure_f8_workspace(ll_layer* h, int M, cudaStream_t st) {
+  if (!h->f8_part) {
+    // Two partial-tile slots per CTA pair.
+    const size_t bytes = static_cast<size_t>(f8_cluster_count(h)) * 2 * 2 * llk::kF8PartFloats * sizeof(float);
+    if (cudaMallocAsync(reinterpret_cast<void**>(&h->f8_part), bytes, st) != cudaSuccess) {
+      cudaGetLastError();
+      h->f8_part = nullptr;
+      return LL_ERR_OOM;
+    }
+  }
+  if (M <= h->ws8_M) return LL_OK;
+  int newM = std::max(M, h->ws8_M * 3 / 2);
+  newM = (newM + 255) / 256 * 256;
+  int *e = nullptr, *cnt = nullptr;
+  uint8_t *a = nullptr, *b = nullptr;
+  const size_t bytes = static_cast<size_t>(newM) * h->K;
+  const size_t ncnt = static_cast<size_t>(newM / 256) * ((h->N + 255) / 256) * 8;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&e), sizeof(int) * newM, st) != cudaSuccess ||
+      cudaMallocAsync(reinterpret_cast<void**>(&a), bytes, st) != cudaSuccess ||
+      cudaMallocAsync(reinterpret_cast<void**>(&b), bytes, st) != cudaSuccess ||
+      cudaMallocAsync(reinterpret_cast<void**>(&cnt), sizeof(int) * ncnt, st) != cudaSuccess ||
+      cudaMemsetAsync(cnt, 0, sizeof(int) * ncnt, st) != cudaSuccess) {
+    cudaGetLastError();
+    if (e) cudaFreeAsync(e, st);
+    if (a) cudaFreeAsync(a, st);
+    if (b) cudaFreeAsync(b, st);
+    if (cnt) cudaFreeAsync(cnt, st);
+    return LL_ERR_OOM;
+  }
+  if (h->e_tok) cudaFreeAsync(h->e_tok, st);
+  if (h->xh) cudaFreeAsync(h->xh, st);
+  if (h->xl) cudaFreeAsync(h->xl, st);
+  if (h->f8_cnt) cudaFreeAsync(h->f8_cnt, st);
+  h->e_tok = e;
+  h->xh = a;
+  h->xl = b;
+  h->f8_cnt = cnt;
+  h->f8_cnt_n = ncnt;
+  h->ws8_M = newM;
+  h->c_M = -1;  // maps over the codes must be rebuilt
+  return LL_OK;
+}
+
+enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM, PATH_F8 };
 
 constexpr int kStreamMaxM = 64;
 constexpr int kPairMaxM = 256;
 
 Path choose_path(const ll_layer* h, int M) {
+  if (h->variant == LL_VARIANT_FP8_SPLIT || h->variant == LL_VARIANT_FP8_ACT) return PATH_F8;
   if (h->variant == LL_VARIANT_TC) return PATH_TC1;
   if (h->variant == LL_VARIANT_TC_PAIR) return PATH_TC2;
   if (h->variant == LL_VARIANT_SMALL) return PATH_SMALL;
@@ -383,6 +470,9 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   // wait for it, so it takes all SMs.
   int budget = h->num_sms;
   if (path == PATH_STREAM) budget = std::max(1, h->num_sms - stream_ctas(h));
+  // Beside the FP8-operand kernel, whose tiles need t only at their end:
+  // half of the SMs.
+  if (path == PATH_F8) budget = std::max(1, h->num_sms / 2);
   int ks = std::max(1, budget / ctas);
   ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);
   if (path == PATH_TC1 && M > 128) ks = plan_tc1(h, M).ks;
@@ -393,26 +483,47 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
 }
 
 // Launches the down-projection; its K splits form one cluster per tile.
+// With lpp.wait_prior it is a programmatic dependent of the kernel before.
 cudaError_t launch_lrdown(const llk::LrDownParams& lpp, const LrPlan& lp, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(lp.m_tiles, lp.r_chunks, lp.ksplit);
   cfg.blockDim = dim3(llk::kLrThreads);
   cfg.dynamicSmemBytes = llk::lr_smem_bytes(lp.rc);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = static_cast<unsigned>(lp.ksplit);
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (lp.ksplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = static_cast<unsigned>(lp.ksplit);
+    ++na;
+  }
+  if (lpp.wait_prior) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = lp.ksplit > 1 ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, llk::ll_lrdown_kernel, lpp);
 }
 
-bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
-  if (h->c_x == x && h->c_yptr == y && h->c_M == M) return true;
+bool build_call_maps(ll_layer* h, const void* x, void* y, int M, bool f8) {
+  if (h->c_x == x && h->c_yptr == y && h->c_M == M && (!f8 || h->c_f8)) return true;
   using namespace llk;
   bool ok = true;
+  if (f8) {
+    constexpr CUtensorMapDataType kU8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    ok &= make_map(&h->c_xh, h->xh, kU8, M, h->K, h->K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->c_xl, h->xl, kU8, M, h->K, h->K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->c_y64, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (h->r_pad > 0) {
+      ok &= make_map(&h->c_thi32, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+      ok &= make_map(&h->c_tlo32, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+    }
+  }
+  h->c_f8 = f8;
   ok &= make_map(&h->c_x128, x, kBF16, M, h->K, 2ull * h->K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&h->c_x256, x, kBF16, M, h->K, 2ull * h->K, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&h->c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -469,6 +580,40 @@ bool build_call_maps(ll_layer* h, const void* x, void* y, int M) {
   return true;
 }
 
+// Data-parallel waves of the FP8-operand kernel before its stream-K tiles.
+// By default every tile is whole and taken from the counter (measured on
+// B200: the stream-K tail's partial sums and the pairs' uneven start times,
+// while the down-projection still holds SMs, cost more than the last
+// partial wave).  LL_FP8_STREAMK=1 in the environment spreads the last
+// partial wave (with the last whole wave when it is short) stream-K.
+int f8_dp_waves(int tiles, int clusters) {
+  static const int sk = [] {
+    const char* e = std::getenv("LL_FP8_STREAMK");
+    return e && e[0] == '1' ? 1 : 0;
+  }();
+  if (!sk) return (tiles + clusters - 1) / clusters;
+  int D = tiles / clusters;
+  const int S = tiles - D * clusters;
+  if (S > 0 && D > 0 && 2 * S < clusters) --D;
+  return D;
+}
+
+// Co-resident clusters of the FP8-operand kernel (asked once per layer).
+int f8_cluster_count(const ll_layer* h) {
+  if (h->f8_clusters > 0) return h->f8_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(h->num_sms);
+  cfg.blockDim = dim3(llk::kF8Threads);
+  cfg.dynamicSmemBytes = llk::f8_smem_bytes();
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, llk::ll_f8_kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = h->num_sms / 2;
+  }
+  h->f8_clusters = std::min(n, h->num_sms / 2);
+  return h->f8_clusters;
+}
+
 int pair_cluster_count(const ll_layer* h) {
   if (h->pair_clusters > 0) return h->pair_clusters;
   cudaLaunchConfig_t cfg = {};
@@ -491,7 +636,11 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   const LrPlan lp = plan_lowrank(h, M);
   int rc = ensure_workspace(h, M, st);
   if (rc != LL_OK) return rc;
-  if (!build_call_maps(h, x, y, M)) return LL_ERR_CUDA;
+  if (path == PATH_F8) {
+    rc = ensure_f8_workspace(h, M, st);
+    if (rc != LL_OK) return rc;
+  }
+  if (!build_call_maps(h, x, y, M, path == PATH_F8)) return LL_ERR_CUDA;
   const Watch watch{h->status, h->timeout_ns};
   int launches = 0;
   const bool prof = h->profiling != 0;
@@ -500,6 +649,18 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     for (cudaEvent_t& e : h->ev)
       if (!e && cudaEventCreate(&e) != cudaSuccess) return LL_ERR_CUDA;
     cudaEventRecord(h->ev[0], st);
+  }
+
+  const int f8_terms = h->variant == LL_VARIANT_FP8_ACT ? 1 : 2;
+  if (path == PATH_F8) {
+    // Per-token exponents and e4m3 codes of x; the down-projection and the
+    // FP8-operand kernel below both read them.
+    const int blocks = std::max(1, std::min((M + 7) / 8, h->num_sms * 8));
+    ll_xsplit_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x), M, h->K, f8_terms, h->e_tok, h->xh,
+                                            h->xl);
+    h->names[launches++] = "ll_xsplit_kernel";
+    if (prof) cudaEventRecord(h->ev[launches], st);
+    if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
   }
 
   if (h->r_pad > 0) {
@@ -520,6 +681,9 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     lpp.tmem_cols = lp.tmem_cols;
     lpp.ksplit = lp.ksplit;
     lpp.kb_per_split = lp.kb_per_split;
+    lpp.e_tok = path == PATH_F8 ? h->e_tok : nullptr;
+    // Beside the split of x, which writes the token exponents it reads.
+    lpp.wait_prior = path == PATH_F8 && !prof ? 1 : 0;
     lpp.watch = watch;
     const cudaError_t lerr = launch_lrdown(lpp, lp, st);
     h->names[launches++] = "ll_lrdown_kernel";
@@ -540,7 +704,42 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   cfg.attrs = attr;
   cfg.numAttrs = overlap ? 1 : 0;
   cudaError_t err;
-  if (path == PATH_STREAM) {
+  if (path == PATH_F8) {
+    F8Params fp;
+    fp.tm_xh = h->c_xh;
+    fp.tm_xl = h->c_xl;
+    fp.tm_q = h->tm_q128;
+    fp.tm_ahi = h->tm_ahi32;
+    fp.tm_alo = h->tm_alo32;
+    fp.tm_thi = h->r_pad > 0 ? h->c_thi32 : h->c_xh;  // unused when r_pad == 0
+    fp.tm_tlo = h->r_pad > 0 ? h->c_tlo32 : h->c_xh;
+    fp.tm_y = h->c_y64;
+    fp.e_tok = h->e_tok;
+    fp.scale = h->scale_eff;
+    fp.bias = h->has_bias ? h->bias : nullptr;
+    fp.part = h->f8_part;
+    fp.cnt = h->f8_cnt;
+    fp.sched = h->sched;
+    fp.M = M;
+    fp.N = h->N;
+    fp.K = h->K;
+    fp.r_pad = h->r_pad;
+    fp.terms = f8_terms;
+    fp.n_ttiles = (M + 255) / 256;
+    fp.n_ftiles = (h->N + 255) / 256;
+    fp.lr_from_primary = overlap ? 1 : 0;
+    fp.watch = watch;
+    // Stream-K over (tile, 128-wide K step) units: one equal range per pair.
+    const long long units = static_cast<long long>(fp.n_ttiles) * fp.n_ftiles * ((h->K + 127) / 128);
+    const int clusters = static_cast<int>(std::max(1LL, std::min<long long>(f8_cluster_count(h), units)));
+    fp.clusters = clusters;
+    fp.dp_waves = f8_dp_waves(fp.n_ttiles * fp.n_ftiles, clusters);
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(kF8Threads);
+    cfg.dynamicSmemBytes = f8_smem_bytes();
+    err = cudaLaunchKernelEx(&cfg, ll_f8_kernel, fp);
+    h->names[launches] = "ll_f8_kernel";
+  } else if (path == PATH_STREAM) {
     StreamParams sp;
     const bool dims3 = h->K % 64 == 0;
     sp.tm_x = h->c_xs;
@@ -767,7 +966,10 @@ ll_handle ll_create(int N, int K, int r, int scale_mode) {
     ok &= make_map(&h->tm_a, h->A, kBF16, N, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&h->tm_ahi, h->Ahi, kBF16, N, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
     ok &= make_map(&h->tm_alo, h->Alo, kBF16, N, h->r_pad, 2ull * h->r_pad, h->klr, 128, sw);
+    ok &= make_map(&h->tm_ahi32, h->Ahi, kBF16, N, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+    ok &= make_map(&h->tm_alo32, h->Alo, kBF16, N, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
   }
+  ok &= make_map(&h->tm_q128, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     free_layer_mem(h);
@@ -783,11 +985,11 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
   g_last_error = LL_OK;
   if (!h || !Q || !scale) return fail(LL_ERR_INVALID_ARG);
   if (h->r > 0 && (!A || !B)) return fail(LL_ERR_INVALID_ARG);
+  if (!aligned(Q, 16) || !aligned(scale, 4) || (bias && !aligned(bias, 2)) ||
+      (h->r > 0 && (!aligned(A, 16) || !aligned(B, 16))))
+    return fail(LL_ERR_INVALID_ARG);
   if (!is_device_ptr(Q) || !is_device_ptr(scale) || (bias && !is_device_ptr(bias)) ||
       (h->r > 0 && (!is_device_ptr(A) || !is_device_ptr(B))))
-    return fail(LL_ERR_INVALID_ARG);
-  if (!aligned(Q, 16) || !aligned(scale, 4) || (bias && !aligned(bias, 2)) ||
-      (h->r > 0 && (!aligned(A, 2) || !aligned(B, 2))))
     return fail(LL_ERR_INVALID_ARG);
   const int N = h->N, K = h->K, r = h->r, rp = h->r_pad;
   const int ns = h->scale_mode == LL_SCALE_PER_ROW ? N : 1;
@@ -834,6 +1036,8 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
       ok &= cudaMalloc(&h->Qf, nq) == cudaSuccess;
       ok &= make_map(&h->tm_qf, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, llk::kBK, 128,
                      CU_TENSOR_MAP_SWIZZLE_64B);
+      ok &= make_map(&h->tm_q128, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
       if (K % 64 == 0) {
         ok &= make_map3(&h->tm_q3, h->Qf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
                         CU_TENSOR_MAP_SWIZZLE_64B);
@@ -849,6 +1053,7 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
     cudaFree(h->Qf);
     h->Qf = h->Q;
     h->tm_qf = h->tm_q;
+    ok &= make_map(&h->tm_q128, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (K % 64 == 0) {
       ok &= make_map3(&h->tm_q3, h->Q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, N, K / 64, K, 64, 64, 128, 4,
                       CU_TENSOR_MAP_SWIZZLE_64B);
@@ -950,8 +1155,7 @@ int ll_reserve(ll_handle h, int max_M) {
 
 int ll_set_variant(ll_handle h, int variant) {
   g_last_error = LL_OK;
-  if (!h || (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC && variant != LL_VARIANT_SMALL &&
-             variant != LL_VARIANT_TC_PAIR && variant != LL_VARIANT_STREAM))
+  if (!h || (variant < LL_VARIANT_AUTO || variant > LL_VARIANT_FP8_ACT))
     return fail(LL_ERR_INVALID_ARG);
   h->variant = variant;
   return LL_OK;
@@ -960,8 +1164,7 @@ int ll_set_variant(ll_handle h, int variant) {
 int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int* kernel, int* tile_tokens, int* lr_splits) {
   g_last_error = LL_OK;
   if (N < 1 || K < 16 || r < 0 || (N % 8) != 0 || (K % 16) != 0 || M < 1 || num_sms < 2 ||
-      (variant != LL_VARIANT_AUTO && variant != LL_VARIANT_TC && variant != LL_VARIANT_SMALL &&
-       variant != LL_VARIANT_TC_PAIR && variant != LL_VARIANT_STREAM))
+      (variant < LL_VARIANT_AUTO || variant > LL_VARIANT_FP8_ACT))
     return fail(LL_ERR_INVALID_ARG);
   if (r > 512) return fail(LL_ERR_UNSUPPORTED);
   // A handle-shaped view holding only what the planning reads.
@@ -989,6 +1192,10 @@ int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int* kernel, i
       kv = LL_VARIANT_STREAM;
       bt = (M + 15) / 16 * 16;
       break;
+    case PATH_F8:
+      kv = variant;
+      bt = 256;
+      break;
     case PATH_SMALL:
       break;
   }
@@ -1011,6 +1218,7 @@ int ll_status(ll_handle h) {
     // A kernel gave up part-way: clear the status and the tile scheduler.
     cudaMemset(h->status, 0, sizeof(int));
     cudaMemset(h->sched, 0, 2 * sizeof(int));
+    if (h->f8_cnt) cudaMemset(h->f8_cnt, 0, sizeof(int) * h->f8_cnt_n);
     cudaDeviceSynchronize();
     return LL_ERR_DEVICE_TIMEOUT;
   }
@@ -1059,6 +1267,27 @@ const char* ll_kernel_name(ll_handle h, int i) {
   return h->names[i];
 }
 
+int ll_quantize_x(const void* x, int M, int K, int terms, int* e_out, void* hi, void* lo, void* stream) {
+  g_last_error = LL_OK;
+  if (M < 0 || K < 16 || (K % 16) != 0 || (terms != 1 && terms != 2)) return fail(LL_ERR_INVALID_ARG);
+  if (M == 0) return LL_OK;
+  if (!x || !e_out || !hi || (terms == 2 && !lo)) return fail(LL_ERR_INVALID_ARG);
+  if (!aligned(x, 16) || !aligned(e_out, 4) || !aligned(hi, 16) || (terms == 2 && !aligned(lo, 16)))
+    return fail(LL_ERR_INVALID_ARG);
+  if (!is_device_ptr(x) || !is_device_ptr(e_out) || !is_device_ptr(hi) || (terms == 2 && !is_device_ptr(lo)))
+    return fail(LL_ERR_INVALID_ARG);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  const int blocks = std::max(1, std::min((M + 7) / 8, sms * 8));
+  llk::ll_xsplit_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x), M, K, terms, e_out, static_cast<uint8_t*>(hi), static_cast<uint8_t*>(lo));
+  if (cudaGetLastError() != cudaSuccess) return fail(LL_ERR_CUDA);
+  return LL_OK;
+}
+
 void ll_destroy(ll_handle h) {
   if (!h) return;
   cudaDeviceSynchronize();
@@ -1085,22 +1314,24 @@ namespace {
 constexpr int kNoAllocMaxDevices = 64;
 
 struct NoAllocDevice {
-  std::once_flag once;
-  int rc = LL_ERR_CUDA;
+  bool ready = false;                // set-up succeeded (a failed set-up is retried by the next call)
   unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
   int num_sms = 0;
 };
 NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+std::mutex g_noalloc_mutex;
 
 // Once per device, with that device current: the scratch address, the SM
-// count and the kernels' shared-memory limits.
+// count and the kernels' shared-memory limits.  Only a successful set-up
+// is kept, so a transient failure does not stick to the device.
 NoAllocDevice* noalloc_setup(int dev, int* rc) {
   if (dev < 0 || dev >= kNoAllocMaxDevices) {
     *rc = LL_ERR_UNSUPPORTED;
     return nullptr;
   }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   NoAllocDevice& d = g_noalloc_dev[dev];
-  std::call_once(d.once, [&d, dev] {
+  if (!d.ready) {
     void* p = nullptr;
     int sms = 0;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr ||
@@ -1110,15 +1341,15 @@ NoAllocDevice* noalloc_setup(int dev, int* rc) {
         cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::lr_smem_bytes(256)) != cudaSuccess) {
       cudaGetLastError();
-      d.rc = LL_ERR_CUDA;
-      return;
+      *rc = LL_ERR_CUDA;
+      return nullptr;
     }
     d.scratch = static_cast<unsigned char*>(p);
     d.num_sms = sms;
-    d.rc = LL_OK;
-  });
-  *rc = d.rc;
-  return d.rc == LL_OK ? &d : nullptr;
+    d.ready = true;
+  }
+  *rc = LL_OK;
+  return &d;
 }
 
 // A per-tensor scale, repeated for each of the N output features.
@@ -1209,6 +1440,8 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
     lpp.tmem_cols = lp.tmem_cols;
     lpp.ksplit = lp.ksplit;
     lpp.kb_per_split = lp.kb_per_split;
+    lpp.e_tok = nullptr;
+    lpp.wait_prior = 0;
     lpp.watch = watch;
     if (launch_lrdown(lpp, lp, st) != cudaSuccess) {
       cudaGetLastError();
@@ -1267,12 +1500,21 @@ extern "C" int ll_forward_noalloc(const void* x, const void* A, const void* B, c
   if (!aligned(x, 16) || !aligned(y, 16) || !aligned(Q, 16) || !aligned(scale, 4) || (bias && !aligned(bias, 2)) ||
       (r > 0 && (!aligned(A, 16) || !aligned(B, 16))))
     return fail(LL_ERR_INVALID_ARG);
-  const char* xb = static_cast<const char*>(x);
-  const char* yb = static_cast<const char*>(y);
-  const size_t xs = static_cast<size_t>(M) * K * 2, ys = static_cast<size_t>(M) * N * 2;
-  if (xb < yb + ys && yb < xb + xs) return fail(LL_ERR_INVALID_ARG);
-  if (!is_device_ptr(x) || !is_device_ptr(y) || !is_device_ptr(Q) || !is_device_ptr(scale) ||
-      (bias && !is_device_ptr(bias)) || (r > 0 && (!is_device_ptr(A) || !is_device_ptr(B))))
+  // y must not overlap any input: the inputs are read in place on every call.
+  const size_t ys = static_cast<size_t>(M) * N * 2;
+  if (overlaps(y, ys, x, static_cast<size_t>(M) * K * 2) || overlaps(y, ys, Q, static_cast<size_t>(N) * K) ||
+      overlaps(y, ys, scale, scale_mode == LL_SCALE_PER_ROW ? 4 * static_cast<size_t>(N) : 4) ||
+      (bias && overlaps(y, ys, bias, 2 * static_cast<size_t>(N))) ||
+      (r > 0 && (overlaps(y, ys, A, 2 * static_cast<size_t>(N) * r) || overlaps(y, ys, B, 2 * static_cast<size_t>(r) * K))))
+    return fail(LL_ERR_INVALID_ARG);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  if (!is_device_ptr_on(x, dev) || !is_device_ptr_on(y, dev) || !is_device_ptr_on(Q, dev) ||
+      !is_device_ptr_on(scale, dev) || (bias && !is_device_ptr_on(bias, dev)) ||
+      (r > 0 && (!is_device_ptr_on(A, dev) || !is_device_ptr_on(B, dev))))
     return fail(LL_ERR_INVALID_ARG);
   const int rc = forward_noalloc(x, A, B, Q, scale, scale_mode, bias, y, M, N, K, r, static_cast<cudaStream_t>(stream));
   return rc == LL_OK ? LL_OK : fail(rc);

@@ -76,8 +76,13 @@ struct LrDownParams {
   int tmem_cols;     // power of two >= rc
   int ksplit;        // number of K splits (gridDim.z; one cluster along z when > 1)
   int kb_per_split;  // 64-wide K steps per split
+  const int* e_tok;  // [M] token exponents: t is written divided by 2^e_tok[m]; nullptr: unscaled
+  int wait_prior;    // 1: e_tok comes from the kernel before (programmatic dependent launch): wait for
+                     // it before the epilogue, and let this kernel's dependents launch only then
   Watch watch;
 };
+
+__device__ __forceinline__ float exp2_int(int e) { return __int_as_float((127 + e) << 23); }
 
 // Ring depth: as many stages as fit in 192 KB (4 to 8): t's reads of x come
 // from HBM, so the more bytes in flight the closer to its bandwidth.
@@ -125,7 +130,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
   int ps = 0, issued = 0;
   uint32_t pph = 0;
   if (threadIdx.x == 0) {
-    pdl_launch_dependents();
+    if (!p.wait_prior) pdl_launch_dependents();
     for (int s = 0; s < n_stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -201,6 +206,11 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
     const int q = warp & 3;
     const int row = 32 * q + lane;
     const int m = m0 + row;
+    if (p.wait_prior) {
+      // The token exponents are written by the kernel before this one.
+      pdl_wait_primary();
+      if (warp == 2 && lane == 0) pdl_launch_dependents();
+    }
     if (__all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.watch, kErrTimeoutEpilogue))) {
       tc_fence_after();
       const bool empty_range = kb_end <= kb_begin;
@@ -218,11 +228,13 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
                 make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
                             __uint_as_float(v[4 * i + 3]));
         } else if (m < p.M) {
+          // exact: a power-of-two scaling of a value far from both ends of the range
+          const float mult = p.e_tok != nullptr ? exp2_int(-p.e_tok[m]) : 1.f;
           uint32_t hi[16], lo[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a = __uint_as_float(v[2 * i]);
-            const float b = __uint_as_float(v[2 * i + 1]);
+            const float a = __uint_as_float(v[2 * i]) * mult;
+            const float b = __uint_as_float(v[2 * i + 1]) * mult;
             const uint16_t ha = to_bf16_bits(a), hb = to_bf16_bits(b);
             hi[i] = static_cast<uint32_t>(ha) | (static_cast<uint32_t>(hb) << 16);
             lo[i] = pack_bf16x2(a - bf16_bits_to_float(ha), b - bf16_bits_to_float(hb));
@@ -245,6 +257,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
     tmem_dealloc(tbase, ncols);
   }
   if (p.ksplit == 1) return;
+  if (p.wait_prior) pdl_wait_primary();  // the reduction below reads the token exponents
 
   // Split K: the CTAs of a cluster hold the partials of one tile; after the
   // cluster barrier, CTA kz sums rows [kz * rpc, (kz + 1) * rpc) of every
@@ -276,6 +289,13 @@ __global__ void __launch_bounds__(kLrThreads, 1) ll_lrdown_kernel(const __grid_c
         acc.z += v[z].z;
         acc.w += v[z].w;
       }
+    if (p.e_tok != nullptr) {
+      const float mult = exp2_int(-p.e_tok[m0 + row]);
+      acc.x *= mult;
+      acc.y *= mult;
+      acc.z *= mult;
+      acc.w *= mult;
+    }
     const uint16_t h0 = to_bf16_bits(acc.x), h1 = to_bf16_bits(acc.y);
     const uint16_t h2 = to_bf16_bits(acc.z), h3 = to_bf16_bits(acc.w);
     uint2 hv, lv;

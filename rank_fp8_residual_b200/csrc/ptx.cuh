@@ -60,25 +60,37 @@ __device__ __forceinline__ uint64_t clock_cycles() {
 
 // Bounded wait on an mbarrier phase.  Returns false (after recording
 // `code` in *w.status) when the phase has not completed within the time
-// limit, or as soon as another thread of the grid has recorded an error,
-// so every role of every CTA drains out instead of spinning.  The fast
-// path only polls; the limit is measured with the SM cycle counter
-// (w.timeout_ns nanoseconds are taken as 2 cycles each, a bound that is
-// at least w.timeout_ns at any SM clock up to 2 GHz).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Watch& w, int code) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+// limit, or when another thread of the grid has recorded an error, so every
+// role of every CTA drains out instead of spinning.  The fast path only
+// polls the barrier: the clock is read once per 256 polls, and the status
+// word in global memory only after a wait has lasted 2^17 cycles (an error
+// is seen within well under a millisecond; a status read on the fast path
+// would put an L2 round trip between a barrier's completion and its
+// waiter).  The limit is measured with the SM cycle counter (w.timeout_ns
+// nanoseconds are taken as 2 cycles each, a bound that is at least
+// w.timeout_ns at any SM clock up to 2 GHz).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity);
+
+template <bool kCluster>
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, const Watch& w, int code) {
   const uint64_t t0 = clock_cycles();
   for (;;) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(a, parity)) return true;
-    if (*reinterpret_cast<volatile int*>(w.status) != 0) return false;
-    if (clock_cycles() - t0 > 2ull * w.timeout_ns) {
+    for (int i = 0; i < 256; ++i)
+      if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
+    const uint64_t dt = clock_cycles() - t0;
+    if (dt > (1ull << 17) && *reinterpret_cast<volatile int*>(w.status) != 0) return false;
+    if (dt > 2ull * w.timeout_ns) {
       atomicCAS(w.status, 0, code);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Watch& w, int code) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  return mbar_wait_slow<false>(a, parity, w, code);
 }
 
 // ----------------------------------------------------------------------- TMA
@@ -326,17 +338,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, const Watch& w, int code) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait_cluster(a, parity)) return true;
-  const uint64_t t0 = clock_cycles();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_cluster(a, parity)) return true;
-    if (*reinterpret_cast<volatile int*>(w.status) != 0) return false;
-    if (clock_cycles() - t0 > 2ull * w.timeout_ns) {
-      atomicCAS(w.status, 0, code);
-      return false;
-    }
-  }
+  return mbar_wait_slow<true>(a, parity, w, code);
 }
 // TMA load into this CTA's shared memory whose completion is signalled on
 // an mbarrier of either CTA of the pair (`mbar` is a cluster address).
@@ -394,6 +396,46 @@ __device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, ui
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Pair MMA on e4m3fn operands (M = 256 across the two CTAs):
+// D (+)= A(smem) * B(smem)^T, e4m3 x e4m3 -> fp32, K = 32 per instruction.
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for tcgen05.mma kind::f8f6f4 with e4m3 A and B
+// (format code 0), fp32 accumulation, both operands K-major.
+__host__ __device__ __forceinline__ constexpr uint32_t idesc_e4m3(int m, int n) {
+  return (1u << 4)                                  // D format: f32
+         | (0u << 7)                                // A format: e4m3
+         | (0u << 10)                               // B format: e4m3
+         | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
+}
+
+// Two fp32 values rounded to e4m3fn (nearest even, saturating at +-448),
+// packed with `lo` in bits 0-7 and `hi` in bits 8-15.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two e4m3fn codes (bits 0-7, 8-15) widened to two fp32 values (exact).
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t v) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
+  float2 r;
+  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(h2));
+  return r;
 }
 
 // Warp-level bf16 MMA m16n8k16 with fp32 accumulation (legacy tensor path).

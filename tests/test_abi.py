@@ -100,3 +100,30 @@ def test_noalloc_argument_checks_need_no_gpu():
     assert f(P, P, P, P, P, 1, P, P, 4, 64, 64, 12, P) == ll.LL_ERR_UNSUPPORTED  # r % 8
     assert f(P, P, P, P, P, 1, P, P, 4, 64, 64, 8, P) == ll.LL_ERR_INVALID_ARG   # null pointers
     assert ll.ll_last_error() == ll.LL_ERR_INVALID_ARG
+
+
+def test_misaligned_pointers_are_rejected_before_any_gpu_work():
+    """The header's alignment rule (16 bytes for x, y, A, B, Q and the e4m3
+    code buffers; 4 for scale and token exponents; 2 for bias) is checked
+    before any CUDA call: fake addresses suffice, no GPU is touched."""
+    import rank_fp8_residual_b200 as ll
+    good = 0x100000
+    bad16 = good + 2
+    base = dict(x=good, A=good, B=good, Q=good, scale=good, bias=good, y=good + 0x800000)
+    for name in ("x", "A", "B", "Q", "y"):
+        a = dict(base, **{name: bad16})
+        with pytest.raises(ll.LLError) as e:
+            ll.ll_forward_noalloc(a["x"], a["A"], a["B"], a["Q"], a["scale"], 1, a["bias"], a["y"],
+                                  64, 256, 256, 32, stream=0)
+        assert e.value.code == ll.LL_ERR_INVALID_ARG, name
+    with pytest.raises(ll.LLError) as e:
+        ll.ll_forward_noalloc(good, good, good, good, good + 2, 1, good, good + 0x800000, 64, 256, 256, 32, stream=0)
+    assert e.value.code == ll.LL_ERR_INVALID_ARG
+    with pytest.raises(ll.LLError) as e:
+        ll.ll_forward_noalloc(good, good, good, good, good, 1, good + 1, good + 0x800000, 64, 256, 256, 32, stream=0)
+    assert e.value.code == ll.LL_ERR_INVALID_ARG
+    for x, e_out, hi, lo in ((bad16, good, good, good), (good, good + 2, good, good), (good, good, bad16, good),
+                             (good, good, good, bad16)):
+        with pytest.raises(ll.LLError) as e:
+            ll.ll_quantize_x(x, 8, 64, 2, e_out, hi, lo, stream=0)
+        assert e.value.code == ll.LL_ERR_INVALID_ARG

@@ -1,9 +1,19 @@
 """Host-side dispatch and tile planning (ll_plan): no GPU needed.
 
-The pins are the measured crossovers and plans recorded in the design
-notes: STREAM up to 64 tokens, CTA pairs up to 256, the one-CTA fused kernel
-above with 256-token tiles at the attention / FFN / sweep shapes.  The
-properties hold for every plan the library can make.
+The pins are measured on one B200 (148 SMs):
+- Dispatch crossovers, from ``python bench.py --suite crossover --rank 64
+  --steps 10 --warmup 3`` (every variant against M on the K = 4096,
+  N = 16384 family, L2 flushed between calls): the streaming kernel is the
+  fastest up to 64 tokens (29.7 us at M = 1 and 64, against 39.9 us and
+  more for the others), the CTA-pair kernel from 96 to 256 tokens (37.9 to
+  39.9 us, against 40.0 to 68.6 us for the 128 x 128 kernel and 42.0 to
+  44.1 us for the one-CTA fused kernel), the one-CTA fused kernel above.
+- Tile plans, from ``python bench.py --workload <name> --steps 50
+  --warmup 5`` per configuration: 256-token tiles with one down-projection
+  split at the attention, FFN and sweep shapes (forward 42.9 us for the
+  attention projection against 47.7 us for the previous 224-token plan).
+
+The properties hold for every plan the library can make.
 """
 import itertools
 
