@@ -11,8 +11,9 @@ Metric: algorithmic TFLOP/s, F = 2*M*(K*N + r*K + r*N) per step.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 device synchronise on both sides; each step is bracketed by CUDA events on
-the launching stream and L2 is flushed (a 256 MiB write) between steps,
-outside the events.  Multi-GPU (torchrun): each rank runs its own batch of
+the launching stream and L2 is flushed between steps, outside the events,
+by reading a 256 MiB buffer (a read leaves clean lines behind, so no
+write-back of the flush lands inside the next timed step).  Multi-GPU (torchrun): each rank runs its own batch of
 M tokens against its own copy of the factors (token-sharded replicas, no
 data-path collective); the reported time is the max over ranks and the
 value counts the tokens of all ranks (weak scaling).
@@ -21,8 +22,13 @@ Also reported on the same JSON line: ``e2e`` (same metric through
 ``ll_forward_host`` with pinned host buffers, the H2D copy of x and the
 D2H copy of y inside each timed step), ``roofline`` for the dominant kernel
 (per-kernel device times from the library's profiling mode), ``clocks``
-(NVML samples taken during the timed region), ``gpu_launches`` and, on
-rank 0 at N=1, ``cpu_baseline`` (the fp64 CPU oracle on a row sample).
+(NVML samples taken during the timed region), ``gpu_launches``, and, on
+rank 0 at N=1, ``cpu_baseline`` (the fp64 CPU oracle on a row sample) and
+``configs``: every layer configuration (tiny, attention, the FFN pair as
+the sum of up and down, the small batches M = 1, 16, 64, the 24 sweep
+points), each device-timed in the same run with its dominant kernel's
+roofline fraction, and the FP8-activation variant beside the bf16 path on
+the large-M configurations.
 
 ``--impl reference`` times the CPU oracle instead (the reference arm of
 this build) on the same workload, metric and unit.
@@ -47,6 +53,21 @@ from synth_inputs import SCALE_PER_ROW, WORKLOADS  # noqa: E402
 
 DEFAULT_WORKLOAD = "attn_m3630_k2048_n2048_r32"
 FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Evicts L2 between timed steps by reading a buffer twice the size of
+    L2 (126 MB on B200).  A read leaves clean lines behind, so evicting them
+    later costs no write-back inside the next timed step."""
+
+    def __init__(self, device):
+        import torch
+        self._buf = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self._out = torch.empty((), dtype=torch.float32, device=device)
+
+    def __call__(self):
+        import torch
+        torch.sum(self._buf, dim=0, out=self._out)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -121,7 +142,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index, period_s=0.002):
+    def __init__(self, device_index, period_s=0.0):
         self.samples = []
         self.reasons = 0
         self.ok = False
@@ -148,7 +169,8 @@ class ClockSampler:
                 self.reasons |= fn(self._h)
             except Exception:
                 pass
-            time.sleep(period)
+            if period > 0:
+                time.sleep(period)
 
     def start(self):
         if self.ok:
@@ -191,6 +213,15 @@ def cpu_baseline(w, budget_s=8.0):
                       f"{dt:.2f} s wall"}
 
 
+def config_of(w, world, variant):
+    """The configuration both arms report (the same dict, so the two lines
+    compare like with like)."""
+    return {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "r": w.r,
+            "scale_mode": "per_row" if w.scale_mode == SCALE_PER_ROW else "per_tensor",
+            "global_tokens": world * w.M, "parallelism": f"token-sharded replicas x{world}",
+            "variant": variant, "l2": "flushed between steps (256 MiB read, outside the step events)"}
+
+
 def run_reference(args, w):
     """Reference arm: the CPU oracle timed step by step on a row sample."""
     rank = int(os.environ.get("RANK", "0"))
@@ -222,14 +253,139 @@ def run_reference(args, w):
         "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "r": w.r,
-                   "scale_mode": "per_row" if w.scale_mode == SCALE_PER_ROW else "per_tensor"},
+        "config": config_of(w, args.gpus, args.variant),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
     return 0
+
+
+VARIANT_NAMES = ("auto", "tc", "tc_pair", "small", "stream", "fp8_split", "fp8_act")
+
+
+def variant_id(ll, name):
+    return getattr(ll, "LL_VARIANT_" + name.upper())
+
+
+def roofline_of(w, kernel_ms, peaks, peak_src, fp8_act=False):
+    """Roofline of the dominant kernel: algorithmic flops (tensor-bound) or
+    bytes (HBM-bound) of that kernel / its event-timed duration.  The fused
+    kernel's work is x Q^T and the up-projection, 2MN(K + r) flops and every
+    compulsory byte but B's (read by the down-projection only).  The peak is
+    the measured bf16 tensor rate, doubled for the one-term FP8 variant (e4m3
+    operands: the nominal fp8 / bf16 ratio), or the measured copy bandwidth."""
+    _, _, main_flops, main_bytes = work_of(w)
+    dom = max(kernel_ms, key=kernel_ms.get)
+    ms = kernel_ms[dom]
+    t_peak = peaks["bf16_tflops"] * (2.0 if fp8_act else 1.0)
+    if main_flops / (t_peak * 1e12) >= main_bytes / (peaks["hbm_gbs"] * 1e9):
+        ach = main_flops / (ms * 1e-3) / 1e12
+        src = ("e4m3 (2 x bf16 burst, nominal ratio)" if fp8_act else "bf16 burst") + f", of {peak_src}"
+        roof = {"bound": "tensor", "achieved": ach, "peak": t_peak, "unit": "TFLOP/s", "frac": ach / t_peak,
+                "peak_source": src}
+    else:
+        ach = main_bytes / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "peak_source": f"copy bandwidth, of {peak_src}"}
+    roof["kernel"] = dom
+    roof["kernel_ms"] = ms
+    return roof
+
+
+def time_forward(ll, h, x, y, M, flush, stream, steps, warmup):
+    """Median device time (ms) of one forward between CUDA events, L2
+    flushed before each, and the per-kernel times of profiled forwards."""
+    import torch
+    ev = []
+    with torch.cuda.stream(stream):
+        for i in range(warmup + steps):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ll.ll_forward(h, x, y, M, stream)
+            b.record(stream)
+            if i >= warmup:
+                ev.append((a, b))
+    torch.cuda.synchronize()
+    st = ll.ll_status(h)
+    if st != ll.LL_OK:
+        raise SystemExit(f"device status: {ll.status_string(st)}")
+    ms = sorted(a.elapsed_time(b) for a, b in ev)
+    ll.ll_set_profiling(h, True)
+    per = {}
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            flush()
+            ll.ll_forward(h, x, y, M, stream)
+            for name, t in ll.ll_kernel_times(h):
+                per.setdefault(name, []).append(t)
+    ll.ll_set_profiling(h, False)
+    torch.cuda.synchronize()
+    return ms[len(ms) // 2], {k: statistics.median(v) for k, v in per.items()}
+
+
+def run_configs(ll, dev, flush, stream, peaks, peak_src, steps=10, warmup=3):
+    """Every layer configuration, device-timed in this run (AUTO dispatch),
+    with the dominant kernel's roofline fraction; the FFN pair also as the
+    sum of up and down; the FP8-activation variant beside the bf16 path on
+    the large-M configurations.  Activations are drawn on the device from a
+    seeded generator; L2 is flushed before every forward."""
+    import torch
+    from synth_inputs import FFN_PAIR, SMALL_BATCH
+    names = (["tiny_m64_k256_n256_r16", "attn_m3630_k2048_n2048_r32"] + list(FFN_PAIR) + list(SMALL_BATCH) +
+             sorted((n for n in WORKLOADS if n.startswith("sweep_")),
+                    key=lambda n: (WORKLOADS[n].K, WORKLOADS[n].N, WORKLOADS[n].r, WORKLOADS[n].M)))
+    fp8_act_on = {"attn_m3630_k2048_n2048_r32"} | set(FFN_PAIR)
+    out, layers = {}, {}
+    for n in names:
+        w = WORKLOADS[n]
+        key = (w.K, w.N, w.r, w.scale_mode, w.scale_value, w.scale_range)
+        if key not in layers:
+            for old in layers.values():
+                old.close()
+            layers.clear()
+            B, A, Q, scale, bias = w.weights(seed=0)
+            layer = ll.LiteLinearLayer(w.N, w.K, w.r, w.scale_mode)
+            layer.set_weights(A.to(dev) if A is not None else None, B.to(dev) if B is not None else None,
+                              Q.to(dev), scale.to(dev), bias.to(dev) if bias is not None else None)
+            layers[key] = layer
+        h = layers[key].handle
+        ll.ll_reserve(h, w.M)
+        g = torch.Generator(device=dev)
+        g.manual_seed(7)
+        x = torch.randn(w.M, w.K, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+        flops, bytes_, _, _ = work_of(w)
+        for vname in ("auto", "fp8_act") if n in fp8_act_on else ("auto",):
+            ll.ll_set_variant(h, variant_id(ll, vname))
+            ms, kms = time_forward(ll, h, x, y, w.M, flush, stream, steps, warmup)
+            roof = roofline_of(w, kms, peaks, peak_src, fp8_act=vname == "fp8_act")
+            key_out = n if vname == "auto" else n + "@fp8_act"
+            out[key_out] = {"us": round(ms * 1e3, 2), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                            "gbs": round(bytes_ / (ms * 1e-3) / 1e9, 1), "kernel": roof["kernel"],
+                            "kernel_us": round(roof["kernel_ms"] * 1e3, 2), "bound": roof["bound"],
+                            "frac": round(roof["frac"], 3),
+                            "kernels_us": {k: round(v * 1e3, 2) for k, v in kms.items()}}
+        ll.ll_set_variant(h, ll.LL_VARIANT_AUTO)
+        del x, y
+    for old in layers.values():
+        old.close()
+    for suffix in ("", "@fp8_act"):
+        up, down = out.get(FFN_PAIR[0] + suffix), out.get(FFN_PAIR[1] + suffix)
+        if up and down:
+            wu, wd = WORKLOADS[FFN_PAIR[0]], WORKLOADS[FFN_PAIR[1]]
+            us = up["us"] + down["us"]
+            fl = work_of(wu)[0] + work_of(wd)[0]
+            mf = work_of(wu)[2] + work_of(wd)[2]
+            kus = up["kernel_us"] + down["kernel_us"]
+            peak = peaks["bf16_tflops"] * (2.0 if suffix else 1.0)
+            out["ffn_pair_sum" + suffix] = {"us": round(us, 2), "tflops": round(fl / (us * 1e-6) / 1e12, 1),
+                                            "kernel_us": round(kus, 2), "bound": "tensor",
+                                            "frac": round(mf / (kus * 1e-6) / 1e12 / peak, 3)}
+    return out
 
 
 def run_page_suite(args):
@@ -243,7 +399,7 @@ def run_page_suite(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.Stream(device=dev)
     steps = max(1, min(args.steps, 30))
     rows, total_ms, total_flops_calls = [], 0.0, 0.0
@@ -266,7 +422,7 @@ def run_page_suite(args):
         ev = []
         with torch.cuda.stream(stream):
             for i in range(args.warmup + steps):
-                flush.zero_()
+                flush()
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record(stream)
@@ -294,7 +450,7 @@ def run_page_suite(args):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"page_microbench_r{args.rank}", "rank": args.rank,
                    "reading": "w1 = 4096 -> 16384, w2 = 16384 -> 4096 (K, N not on the page)",
-                   "l2": "flushed between calls (256 MiB write, outside the events)", "rows": rows},
+                   "l2": "flushed between calls (256 MiB read, outside the events)", "rows": rows},
         "tflops_weighted": total_flops_calls / (total_ms * 1e-3) / 1e12,
         "vs_baseline": None,
     }
@@ -313,7 +469,7 @@ def run_crossover_suite(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.Stream(device=dev)
     K, N, r = 4096, 16384, args.rank
     B, A, Q, scale, bias = make_weights(K, N, r, seed=0)
@@ -340,7 +496,7 @@ def run_crossover_suite(args):
             ev = []
             with torch.cuda.stream(stream):
                 for i in range(args.warmup + steps):
-                    flush.zero_()
+                    flush()
                     a = torch.cuda.Event(enable_timing=True)
                     b = torch.cuda.Event(enable_timing=True)
                     a.record(stream)
@@ -376,8 +532,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="auto",
-                    choices=["auto", "tc", "tc_pair", "small", "stream", "fp8_split", "fp8_act"],
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration timings")
+    ap.add_argument("--variant", default="auto", choices=list(VARIANT_NAMES),
                     help="kernel variant (auto picks by token count)")
     ap.add_argument("--suite", default=None, choices=["page", "crossover"],
                     help="page: the README's LTX-Video FFN shapes, count-weighted total; "
@@ -415,13 +571,11 @@ def main():
                       inp.Q.to(dev), inp.scale.to(dev),
                       inp.bias.to(dev) if inp.bias is not None else None)
     h = layer.handle
-    ll.ll_set_variant(h, {"auto": ll.LL_VARIANT_AUTO, "tc": ll.LL_VARIANT_TC, "tc_pair": ll.LL_VARIANT_TC_PAIR,
-                          "small": ll.LL_VARIANT_SMALL, "stream": ll.LL_VARIANT_STREAM,
-                          "fp8_split": ll.LL_VARIANT_FP8_SPLIT, "fp8_act": ll.LL_VARIANT_FP8_ACT}[args.variant])
+    ll.ll_set_variant(h, variant_id(ll, args.variant))
     ll.ll_reserve(h, w.M)
     x = inp.x.to(dev)
     y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.Stream(device=dev)
     flops, bytes_, main_flops, main_bytes = work_of(w)
 
@@ -433,7 +587,7 @@ def main():
     # --------------------------------------------------- device-timed steps
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.zero_()
+            flush()
             ll.ll_forward(h, x, y, w.M, stream)
         ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -443,7 +597,7 @@ def main():
         torch.cuda.synchronize()
         sampler.start()
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             ev0[i].record(stream)
             ll.ll_forward(h, x, y, w.M, stream)
             ev1[i].record(stream)
@@ -470,7 +624,7 @@ def main():
         barrier()
         torch.cuda.synchronize()
         for i in range(e2e_steps):
-            flush.zero_()
+            flush()
             e0[i].record(stream)
             ll.ll_forward_host(h, xh.data_ptr(), yh.data_ptr(), w.M, stream)
             e1[i].record(stream)
@@ -485,7 +639,7 @@ def main():
     per_kernel = {}
     with torch.cuda.stream(stream):
         for i in range(prof_steps + 2):
-            flush.zero_()
+            flush()
             ll.ll_forward(h, x, y, w.M, stream)
             if i >= 2:
                 for name, ms in ll.ll_kernel_times(h):
@@ -497,17 +651,7 @@ def main():
     dom_ms = max_over_ranks(kernel_ms[dom])
 
     peaks, peak_src = load_peaks()
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if main_flops / main_bytes >= ridge:
-        ach = main_flops / (dom_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"], "peak_source": f"bf16 burst, of {peak_src}"}
-    else:
-        ach = main_bytes / (dom_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"], "peak_source": f"copy bandwidth, of {peak_src}"}
-    roof["kernel"] = dom
-    roof["kernel_ms"] = dom_ms
+    roof = roofline_of(w, dict(kernel_ms, **{dom: dom_ms}), peaks, peak_src, fp8_act=args.variant == "fp8_act")
     roof["traffic"] = recorded_traffic(dom, w.name)
     roof["kernel_ms_all"] = kernel_ms
 
@@ -515,13 +659,11 @@ def main():
         "metric": "ll_forward TFLOP/s (algorithmic)",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "r": w.r,
-                   "scale_mode": "per_row" if w.scale_mode == SCALE_PER_ROW else "per_tensor",
-                   "global_tokens": world * w.M, "parallelism": f"token-sharded replicas x{world}",
-                   "variant": args.variant,
-                   "l2": "flushed between steps (256 MiB write, outside the step events)",
-                   "hbm_gbs_algorithmic": world * args.steps * bytes_ / (total_ms * 1e-3) / 1e9},
+        "scaling": "weak", "vs_baseline": None,
+        # the arithmetic of the dominant kernel: bf16 x bf16 MMAs, or e4m3 x e4m3 (FP8-operand kernel)
+        "dtype": "e4m3" if roof["kernel"] == "ll_f8_kernel" else "bf16", "data": "synthetic",
+        "config": config_of(w, world, args.variant),
+        "hbm_gbs_algorithmic": world * args.steps * bytes_ / (total_ms * 1e-3) / 1e9,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": 2 * w.M * w.K,
                 "d2h_bytes_per_step": 2 * w.M * w.N, "steps": e2e_steps,
                 "api": "ll_forward_host (pinned host buffers)"},
@@ -529,9 +671,11 @@ def main():
         "roofline": roof,
         "clocks": sampler.summary(),
     }
+    layer.close()
+    if rank == 0 and world == 1 and not args.no_configs:
+        line["configs"] = run_configs(ll, dev, flush, stream, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
-    layer.close()
     if world > 1:
         replicas.barrier()
         replicas.finalize()

@@ -140,10 +140,14 @@ int ll_forward(ll_handle h, const void *x, void *y, int M, void *stream);
 /* No counterpart on the pages: the forward from host memory.
  *
  * ll_forward on HOST buffers: copies x (host, bf16 [M, K]) to the device,
- * runs the forward and copies y back to the host (bf16 [M, N]), all on
- * `stream`.  Pinned host buffers make the copies asynchronous; the caller
- * synchronises the stream before reading y.  Device staging buffers are
- * handle-owned and grown on demand. */
+ * runs the forward and copies y back to the host (bf16 [M, N]).  The rows
+ * go in up to four chunks of whole 256-token tiles, so that the copy of
+ * one chunk into the device, the forward of the one before and the copy
+ * out of the one before that overlap (two handle-owned copy streams; the
+ * forwards run on `stream`, which waits for the last copy out).  Pinned
+ * host buffers make the copies asynchronous; the caller synchronises
+ * `stream` once before reading y.  Device staging buffers are
+ * handle-owned and grown on demand.  Errors as ll_forward. */
 int ll_forward_host(ll_handle h, const void *x_host, void *y_host, int M, void *stream);
 
 /* No counterpart on the pages.  Pre-size the workspace for forwards of up

@@ -157,10 +157,14 @@ struct ll_layer {
   CUtensorMap c_xh, c_xl, c_thi32, c_tlo32, c_y64;  // per-call maps of the FP8-operand kernel
   bool c_f8 = false;                           // the per-call FP8 maps are built
   mutable int f8_clusters = 0;                 // co-resident clusters of the FP8-operand kernel
-  // host-buffer forward staging
+  // host-buffer forward staging: device copies of x and y, and two copy
+  // streams (host to device, device to host) that overlap the chunks' copies
+  // with the forwards on the caller's stream
   void* dx = nullptr;
   void* dy = nullptr;
   size_t dx_bytes = 0, dy_bytes = 0;
+  cudaStream_t cin = nullptr, cout = nullptr;
+  cudaEvent_t hev[2 * 8 + 2] = {};  // start, copy-in done [8], forward done [8], copy-out done
   // weight tensor maps
   CUtensorMap tm_q, tm_qf, tm_a, tm_ahi, tm_alo, tm_b;
   int b_box = 0;
@@ -197,6 +201,10 @@ namespace {
 void free_layer_mem(ll_layer* h) {
   for (cudaEvent_t& e : h->ev)
     if (e) cudaEventDestroy(e);
+  for (cudaEvent_t& e : h->hev)
+    if (e) cudaEventDestroy(e);
+  if (h->cin) cudaStreamDestroy(h->cin);
+  if (h->cout) cudaStreamDestroy(h->cout);
   if (h->Qf && h->Qf != h->Q) cudaFree(h->Qf);
   cudaFree(h->Q);
   cudaFree(h->A);
@@ -320,6 +328,16 @@ int ensure_f8_workspace(ll_layer* h, int M, cudaStream_t st) {
 
 enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM, PATH_F8 };
 
+// Where the two-term FP8-operand kernel beats the one-CTA exact-widening
+// kernel for M > 256.  Its split of x costs 2MK bytes each way against a
+// GEMM of 2MNK flops, so it wins on wide layers.  Measured forward times on
+// B200 (us, exact-widening / two-term): N = 4K: 3630 x 2048 -> 8192 122 / 101,
+// 1024 x 4096 -> 16384 122 / 108, 16384 x 4096 -> 16384 1727 / 1470;
+// N = K: 4096 x 4096 -> 4096 124 / 118, 16384 x 4096 -> 4096 450 / 415,
+// 1024 x 4096 -> 4096 40 / 63, 3630 x 2048 -> 2048 42 / 54;
+// N = K / 4: 3630 x 8192 -> 2048 118 / 169, 9800 x 16384 -> 4096 1071 / 1112.
+bool fp8_split_wins(int N, int K, int M) { return N >= 2 * K || (N >= K && M >= 4096); }
+
 constexpr int kStreamMaxM = 64;
 constexpr int kPairMaxM = 256;
 
@@ -332,8 +350,10 @@ Path choose_path(const ll_layer* h, int M) {
   if (M <= kStreamMaxM) return PATH_STREAM;
   // Measured on the K = 4096, N = 16384 family: the CTA-pair kernel with
   // its narrow tiles beats the 128 x 128 and one-CTA kernels up to 256
-  // tokens; above, the one-CTA kernel with its joint plan.
-  return M > kPairMaxM ? PATH_TC1 : PATH_TC2;
+  // tokens; above, the one-CTA kernel with its joint plan, except where the
+  // FP8-operand kernel is faster.
+  if (M <= kPairMaxM) return PATH_TC2;
+  return fp8_split_wins(h->N, h->K, M) ? PATH_F8 : PATH_TC1;
 }
 
 // CTAs of the streaming kernel: one per 128-feature tile, at most one per SM.
@@ -728,6 +748,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     fp.n_ttiles = (M + 255) / 256;
     fp.n_ftiles = (h->N + 255) / 256;
     fp.lr_from_primary = overlap ? 1 : 0;
+    fp.withhold = h->withhold;
     fp.watch = watch;
     // Stream-K over (tile, 128-wide K step) units: one equal range per pair.
     const long long units = static_cast<long long>(fp.n_ttiles) * fp.n_ftiles * ((h->K + 127) / 128);
@@ -1114,7 +1135,17 @@ int ll_forward_host(ll_handle h, const void* x_host, void* y_host, int M, void* 
   if (!h->ready) return fail(LL_ERR_NOT_READY);
   if (M == 0) return LL_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t xs = static_cast<size_t>(M) * h->K * 2, ys = static_cast<size_t>(M) * h->N * 2;
+  const size_t xrow = static_cast<size_t>(h->K) * 2, yrow = static_cast<size_t>(h->N) * 2;
+  const size_t xs = static_cast<size_t>(M) * xrow, ys = static_cast<size_t>(M) * yrow;
+  if (!h->cin) {
+    bool ok = cudaStreamCreateWithFlags(&h->cin, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->cout, cudaStreamNonBlocking) == cudaSuccess;
+    for (cudaEvent_t& e : h->hev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return fail(LL_ERR_CUDA);
+    }
+  }
   if (xs > h->dx_bytes) {
     void* p = nullptr;
     if (cudaMallocAsync(&p, xs, st) != cudaSuccess) { cudaGetLastError(); return fail(LL_ERR_OOM); }
@@ -1129,13 +1160,49 @@ int ll_forward_host(ll_handle h, const void* x_host, void* y_host, int M, void* 
     h->dy = p;
     h->dy_bytes = ys;
   }
-  if (cudaMemcpyAsync(h->dx, x_host, xs, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+  // Chunks of whole 256-token tiles: the copy of chunk i + 1 into the
+  // device, the forward of chunk i and the copy of chunk i - 1 out run at
+  // the same time (the two copy directions on their own streams).  The
+  // caller's stream waits for the last copy out, so synchronising it once
+  // still covers the whole call.
+  const int n_chunks = M >= 2048 ? 4 : (M >= 512 ? 2 : 1);
+  const int rows = (M + n_chunks * 256 - 1) / (n_chunks * 256) * 256;
+  cudaEvent_t* ev_in = h->hev + 1;
+  cudaEvent_t* ev_fwd = h->hev + 1 + 8;
+  cudaEvent_t ev_done = h->hev[2 * 8 + 1];
+  if (cudaEventRecord(h->hev[0], st) != cudaSuccess || cudaStreamWaitEvent(h->cin, h->hev[0], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(h->cout, h->hev[0], 0) != cudaSuccess) {
     cudaGetLastError();
     return fail(LL_ERR_CUDA);
   }
-  int rc = forward_device(h, h->dx, h->dy, M, st);
-  if (rc != LL_OK) return fail(rc);
-  if (cudaMemcpyAsync(y_host, h->dy, ys, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+  int n = 0;
+  for (int m0 = 0; m0 < M; m0 += rows, ++n) {
+    const int mi = std::min(rows, M - m0);
+    if (cudaMemcpyAsync(static_cast<char*>(h->dx) + m0 * xrow, static_cast<const char*>(x_host) + m0 * xrow,
+                        mi * xrow, cudaMemcpyHostToDevice, h->cin) != cudaSuccess ||
+        cudaEventRecord(ev_in[n], h->cin) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(LL_ERR_CUDA);
+    }
+  }
+  n = 0;
+  for (int m0 = 0; m0 < M; m0 += rows, ++n) {
+    const int mi = std::min(rows, M - m0);
+    if (cudaStreamWaitEvent(st, ev_in[n], 0) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(LL_ERR_CUDA);
+    }
+    const int rc = forward_device(h, static_cast<char*>(h->dx) + m0 * xrow, static_cast<char*>(h->dy) + m0 * yrow,
+                                  mi, st);
+    if (rc != LL_OK) return fail(rc);
+    if (cudaEventRecord(ev_fwd[n], st) != cudaSuccess || cudaStreamWaitEvent(h->cout, ev_fwd[n], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<char*>(y_host) + m0 * yrow, static_cast<char*>(h->dy) + m0 * yrow, mi * yrow,
+                        cudaMemcpyDeviceToHost, h->cout) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(LL_ERR_CUDA);
+    }
+  }
+  if (cudaEventRecord(ev_done, h->cout) != cudaSuccess || cudaStreamWaitEvent(st, ev_done, 0) != cudaSuccess) {
     cudaGetLastError();
     return fail(LL_ERR_CUDA);
   }
@@ -1193,7 +1260,7 @@ int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int* kernel, i
       bt = (M + 15) / 16 * 16;
       break;
     case PATH_F8:
-      kv = variant;
+      kv = variant == LL_VARIANT_FP8_ACT ? LL_VARIANT_FP8_ACT : LL_VARIANT_FP8_SPLIT;
       bt = 256;
       break;
     case PATH_SMALL:

@@ -190,6 +190,7 @@ struct F8Params {
   int clusters;          // CTA pairs of the grid
   int dp_waves;          // data-parallel waves of whole tiles before the stream-K tiles
   int lr_from_primary;   // 1: t' is written by the preceding kernel
+  int withhold;          // debug: the producers issue nothing, so every consumer's wait runs out
   Watch watch;
 };
 
@@ -388,6 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
       F8Sched sch(sp, cid);
       F8Seg g;
       while (ok && sch.next(g, tile_full, tile_empty, tile_slot, p.watch, kErrTimeoutProducer, false)) {
+        if (p.withhold) { ok = false; break; }  // debug: no loads, the consumers time out
         int tt, ft;
         f8_tile_coords(p, g.T, tt, ft);
         const int t0 = tt * 256 + 128 * static_cast<int>(rank);

@@ -17,7 +17,8 @@ from llgpu import DeviceLayer, check
 pytestmark = pytest.mark.gpu
 
 CASES = [(ll.LL_VARIANT_TC, 600), (ll.LL_VARIANT_SMALL, 100), (ll.LL_VARIANT_STREAM, 40),
-         (ll.LL_VARIANT_TC_PAIR, 600), (ll.LL_VARIANT_AUTO, 3000)]
+         (ll.LL_VARIANT_TC_PAIR, 600), (ll.LL_VARIANT_AUTO, 3000), (ll.LL_VARIANT_FP8_SPLIT, 600),
+         (ll.LL_VARIANT_FP8_ACT, 300)]
 
 
 @pytest.mark.parametrize("variant,M", CASES)
@@ -35,6 +36,7 @@ def test_withheld_loads_time_out_and_the_handle_recovers(variant, M):
         ll.ll_set_debug(d.h, False, 2_000_000_000)
         for _ in range(2):  # the counters the timed-out launch used are back at zero
             y2 = d.forward(inp.x)
-            check(y2.cpu(), oracle.forward_inputs(inp), what=f"after timeout, variant {variant}")
+            mode = oracle.FP8ACT if variant == ll.LL_VARIANT_FP8_ACT else oracle.EXACT
+            check(y2.cpu(), oracle.forward_inputs(inp, mode=mode), what=f"after timeout, variant {variant}")
     finally:
         d.close()

@@ -12,6 +12,12 @@ The pins are measured on one B200 (148 SMs):
   --warmup 5`` per configuration: 256-token tiles with one down-projection
   split at the attention, FFN and sweep shapes (forward 42.9 us for the
   attention projection against 47.7 us for the previous 224-token plan).
+- The FP8-operand two-term kernel above 256 tokens where N >= 2K, or
+  N >= K with M >= 4096, from forward times measured per variant with L2
+  flushed between calls (us, exact-widening / two-term): 3630 x 2048 ->
+  8192 122 / 101; 1024 x 4096 -> 16384 122 / 108; 4096 x 4096 -> 4096
+  124 / 118; 1024 x 4096 -> 4096 40 / 63; 3630 x 2048 -> 2048 42 / 54;
+  3630 x 8192 -> 2048 118 / 169; 9800 x 16384 -> 4096 1071 / 1112.
 
 The properties hold for every plan the library can make.
 """
@@ -24,17 +30,21 @@ import rank_fp8_residual_b200 as ll
 SMS = 148
 
 
-@pytest.mark.parametrize("N,K,r,M", [
-    (2048, 2048, 32, 3630),     # attention projection
-    (8192, 2048, 64, 3630),     # FFN up
-    (2048, 8192, 64, 3630),     # FFN down
-    (16384, 4096, 64, 8192),    # sweep point
+@pytest.mark.parametrize("N,K,r,M,kernel", [
+    (2048, 2048, 32, 3630, ll.LL_VARIANT_TC),           # attention projection
+    (8192, 2048, 64, 3630, ll.LL_VARIANT_FP8_SPLIT),    # FFN up
+    (2048, 8192, 64, 3630, ll.LL_VARIANT_TC),           # FFN down
+    (16384, 4096, 64, 8192, ll.LL_VARIANT_FP8_SPLIT),   # sweep point
+    (4096, 4096, 64, 1024, ll.LL_VARIANT_TC),           # sweep point, N = K, M < 4096
+    (4096, 4096, 64, 4096, ll.LL_VARIANT_FP8_SPLIT),    # sweep point, N = K, M >= 4096
+    (4096, 16384, 64, 9800, ll.LL_VARIANT_TC),          # README benchmark w2
 ])
-def test_large_m_plans(N, K, r, M):
-    kernel, bt, ks = ll.ll_plan(N, K, r, M, SMS)
-    assert kernel == ll.LL_VARIANT_TC
+def test_large_m_plans(N, K, r, M, kernel):
+    got, bt, ks = ll.ll_plan(N, K, r, M, SMS)
+    assert got == kernel
     assert bt == 256
-    assert ks == 1
+    if kernel == ll.LL_VARIANT_TC:
+        assert ks == 1
 
 
 @pytest.mark.parametrize("M", [1, 16, 33, 64])
@@ -47,8 +57,12 @@ def test_small_batch_streams(M):
 
 def test_auto_crossovers():
     for M, want in [(64, ll.LL_VARIANT_STREAM), (65, ll.LL_VARIANT_TC_PAIR), (256, ll.LL_VARIANT_TC_PAIR),
-                    (257, ll.LL_VARIANT_TC), (4096, ll.LL_VARIANT_TC)]:
+                    (257, ll.LL_VARIANT_FP8_SPLIT), (4096, ll.LL_VARIANT_FP8_SPLIT)]:
         assert ll.ll_plan(16384, 4096, 64, M, SMS)[0] == want, M
+    for M, want in [(257, ll.LL_VARIANT_TC), (4095, ll.LL_VARIANT_TC), (4096, ll.LL_VARIANT_FP8_SPLIT)]:
+        assert ll.ll_plan(4096, 4096, 64, M, SMS)[0] == want, M
+    for M in (257, 3630, 16384):
+        assert ll.ll_plan(2048, 8192, 64, M, SMS)[0] == ll.LL_VARIANT_TC, M
 
 
 def test_forced_variants():
@@ -67,8 +81,10 @@ def test_plan_properties():
     Ms = (1, 63, 64, 65, 128, 129, 256, 257, 1000, 3630, 16384)
     for N, K, r, M in itertools.product(Ns, Ks, rs, Ms):
         kernel, bt, ks = ll.ll_plan(N, K, r, M, SMS)
-        assert kernel in (ll.LL_VARIANT_TC, ll.LL_VARIANT_TC_PAIR, ll.LL_VARIANT_STREAM)
-        if kernel == ll.LL_VARIANT_TC:
+        assert kernel in (ll.LL_VARIANT_TC, ll.LL_VARIANT_TC_PAIR, ll.LL_VARIANT_STREAM, ll.LL_VARIANT_FP8_SPLIT)
+        if kernel == ll.LL_VARIANT_FP8_SPLIT:
+            assert bt == 256 and M > 256 and (N >= 2 * K or (N >= K and M >= 4096))
+        elif kernel == ll.LL_VARIANT_TC:
             assert bt % 32 == 0 and 128 <= bt <= 256
         elif kernel == ll.LL_VARIANT_TC_PAIR:
             assert bt % 32 == 0 and 32 <= bt <= 256
@@ -97,5 +113,7 @@ def test_plan_rejects_bad_arguments():
         ll.ll_plan(4096, 4096, 64, 64, 1)         # num_sms < 2
     with pytest.raises(ll.LLError):
         ll.ll_plan(4096, 4096, 64, 64, SMS, 9)    # unknown variant
+    for v in (ll.LL_VARIANT_FP8_SPLIT, ll.LL_VARIANT_FP8_ACT):
+        assert ll.ll_plan(4096, 4096, 64, 100, SMS, v)[0] == v
     with pytest.raises(ll.LLError):
         ll.ll_plan(4096, 4096, 513, 64, SMS)      # r > 512
