@@ -53,6 +53,9 @@ def lib():
         L.llo_enc_e4m3_rne.argtypes = [ctypes.c_double]
         L.llo_token_exp.restype = ctypes.c_int
         L.llo_token_exp.argtypes = [ctypes.c_double]
+        L.llo_residual_quant.restype = ctypes.c_int
+        L.llo_residual_quant.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
         L.llo_quant_x.restype = ctypes.c_int
         L.llo_quant_x.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -97,6 +100,28 @@ def quant_x(x, terms: int):
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return e, hi, lo
+
+
+def residual_quant(W, A, B, scale_mode):
+    """The residual quantisation of the decomposition step: W, A, B as bf16
+    bits (uint16 [N, K], [N, r] or None, [r, K] or None).  Returns
+    (Q uint8 [N, K], scale float32 [N] or [1])."""
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    N, K = W.shape
+    if A is None or B is None:
+        r = 0
+    else:
+        A = np.ascontiguousarray(A, dtype=np.uint16)
+        B = np.ascontiguousarray(B, dtype=np.uint16)
+        r = A.shape[1]
+        assert A.shape == (N, r) and B.shape == (r, K)
+    Q = np.zeros((N, K), dtype=np.uint8)
+    scale = np.zeros(N if scale_mode == 1 else 1, dtype=np.float32)
+    rc = lib().llo_residual_quant(N, K, r, _ptr(W), _ptr(A) if r else None, _ptr(B) if r else None,
+                                  int(scale_mode), _ptr(Q), _ptr(scale))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return Q, scale
 
 
 def num_threads() -> int:

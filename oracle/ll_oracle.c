@@ -224,6 +224,77 @@ int llo_quant_x(int M, int K, const uint16_t *x, int terms, int *e_out, uint8_t 
 }
 
 /*
+ * The residual quantisation of the decomposition step (LiteLinear README,
+ * "Usage": LiteLinear.from_dense, an SVD-based decomposition; the MoDeGPT
+ * compressor's _decompose_single keeps U_r S_r and V_r^T as the two
+ * factors).  Given W [N][K] and the bf16 factors A [N][r], B [r][K]:
+ *
+ *   R[n][k]  = W[n][k] - sum_j A[n][j] * B[j][k]      (binary64, j in order)
+ *   amax     = max_k |R[n][k]|  (per row)  or  max over all of R (per tensor)
+ *   scale    = amax / 448, rounded to binary32 (0 when amax == 0)
+ *   Q[n][k]  = e4m3fn code nearest to (binary32)(R[n][k] / scale), ties to
+ *              even, saturating at 448; 0 where scale == 0
+ *
+ * The pages do not state how the residual's scale is chosen; the plainest
+ * reading maps each row's largest magnitude to the largest e4m3fn value.
+ * The rounding steps are fixed so that the decision of every code is taken
+ * in the same precision wherever it is computed.  Writes Q [N][K] and
+ * scale [N] (per row) or [1] (per tensor).  Returns 0, or -1 on bad
+ * arguments.
+ */
+int llo_residual_quant(int N, int K, int r, const uint16_t *W, const uint16_t *A, const uint16_t *B,
+                       int scale_mode, uint8_t *Q, float *scale)
+{
+    if (N < 0 || K < 0 || r < 0 || (N > 0 && K > 0 && (!W || !Q)) || !scale ||
+        (r > 0 && N > 0 && K > 0 && (!A || !B)))
+        return -1;
+    if (scale_mode != LLO_SCALE_PER_TENSOR && scale_mode != LLO_SCALE_PER_ROW)
+        return -1;
+    double pos[0x7F];
+    e4m3_positive_values(pos);
+    double *R = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1) * (size_t)(K > 0 ? K : 1));
+    if (!R)
+        return -1;
+    double gmax = 0.0;
+    for (int n = 0; n < N; ++n) {
+        for (int k = 0; k < K; ++k) {
+            double acc = 0.0;
+            for (int j = 0; j < r; ++j)
+                acc = acc + llo_dec_bf16(A[(size_t)n * r + j]) * llo_dec_bf16(B[(size_t)j * K + k]);
+            double v = llo_dec_bf16(W[(size_t)n * K + k]) - acc;
+            R[(size_t)n * K + k] = v;
+            if (fabs(v) > gmax)
+                gmax = fabs(v);
+        }
+    }
+    if (scale_mode == LLO_SCALE_PER_TENSOR)
+        scale[0] = (float)(gmax / 448.0);
+    for (int n = 0; n < N; ++n) {
+        float s;
+        if (scale_mode == LLO_SCALE_PER_ROW) {
+            double amax = 0.0;
+            for (int k = 0; k < K; ++k)
+                if (fabs(R[(size_t)n * K + k]) > amax)
+                    amax = fabs(R[(size_t)n * K + k]);
+            s = (float)(amax / 448.0);
+            scale[n] = s;
+        } else {
+            s = scale[0];
+        }
+        for (int k = 0; k < K; ++k) {
+            uint8_t c = 0;
+            if (s != 0.0f) {
+                float u = (float)(R[(size_t)n * K + k] / (double)s);
+                c = enc_e4m3_search((double)u, pos);
+            }
+            Q[(size_t)n * K + k] = c;
+        }
+    }
+    free(R);
+    return 0;
+}
+
+/*
  * The forward pass for the rows listed in `rows` (or all M rows when
  * rows == NULL), written out as the definition:
  *
