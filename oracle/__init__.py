@@ -171,12 +171,38 @@ def forward(x, B, A, Q, scale, scale_mode, bias=None, mode=EXACT, rows=None):
     return y
 
 
-def forward_inputs(inp, mode=EXACT, rows=None):
-    """forward() on a synth_inputs.LayerInputs."""
+EPILOGUE_NONE = 0
+EPILOGUE_GELU_TANH = 1
+EPILOGUE_GEGLU_TANH = 2
+
+
+def gelu_tanh(v: np.ndarray) -> np.ndarray:
+    """GELU in its tanh form, v / 2 * (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))
+    (the approximation the LTX feed-forward's GELU uses), in binary64."""
+    return 0.5 * v * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (v + 0.044715 * v ** 3)))
+
+
+def apply_epilogue(y: np.ndarray, epilogue: int) -> np.ndarray:
+    """The fused activation on the layer's output y [rows, N]: none, GELU of
+    every element, or GEGLU: h * gelu(g) with h = y[:, :N/2], g = y[:, N/2:]
+    (the LiteLinear README's GEGLU projection, "Usage": replace_activation_proj_)."""
+    if epilogue == EPILOGUE_NONE:
+        return y
+    if epilogue == EPILOGUE_GELU_TANH:
+        return gelu_tanh(y)
+    if epilogue == EPILOGUE_GEGLU_TANH:
+        n = y.shape[1] // 2
+        return y[:, :n] * gelu_tanh(y[:, n:])
+    raise ValueError("unknown epilogue")
+
+
+def forward_inputs(inp, mode=EXACT, rows=None, epilogue=EPILOGUE_NONE):
+    """forward() on a synth_inputs.LayerInputs, then the epilogue activation."""
     from synth_inputs import to_numpy_bits
-    return forward(to_numpy_bits(inp.x), to_numpy_bits(inp.B), to_numpy_bits(inp.A),
-                   to_numpy_bits(inp.Q), to_numpy_bits(inp.scale), inp.scale_mode,
-                   to_numpy_bits(inp.bias), mode=mode, rows=rows)
+    y = forward(to_numpy_bits(inp.x), to_numpy_bits(inp.B), to_numpy_bits(inp.A),
+                to_numpy_bits(inp.Q), to_numpy_bits(inp.scale), inp.scale_mode,
+                to_numpy_bits(inp.bias), mode=mode, rows=rows)
+    return apply_epilogue(y, epilogue)
 
 
 def tolerance_bound(y_ref: np.ndarray, rms: float | None = None) -> np.ndarray:
