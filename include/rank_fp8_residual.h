@@ -154,6 +154,28 @@ int ll_forward_host(ll_handle h, const void *x_host, void *y_host, int M, void *
  * to max_M rows (synchronous). */
 int ll_reserve(ll_handle h, int max_M);
 
+/* Activation fused into the epilogue (ll_set_epilogue).  The LTX-Video
+ * transformers the LiteLinear README converts wrap the first linear of each
+ * feed-forward in a GEGLU ("Usage": replace_activation_proj_ routes the
+ * GEGLU's projection through LiteLinear): proj(x) is split into a value
+ * half h and a gate half g, and the block computes h * gelu(g), with GELU
+ * in its tanh form gelu(v) = v / 2 * (1 + tanh(sqrt(2/pi) (v + 0.044715
+ * v^3))).  LL_EPILOGUE_GELU_TANH applies gelu to every output;
+ * LL_EPILOGUE_GEGLU_TANH returns y[m, j] = h[m, j] * gelu(g[m, j]) with
+ * h = outputs 0 .. N/2 - 1 and g = outputs N/2 .. N - 1 of the formula, so
+ * y is [M, N/2]. */
+enum { LL_EPILOGUE_NONE = 0, LL_EPILOGUE_GELU_TANH = 1, LL_EPILOGUE_GEGLU_TANH = 2 };
+
+/* Select the epilogue activation (no counterpart on the pages beyond the
+ * GEGLU above).  The activation is applied to the fp32 result before its
+ * one rounding to bf16.  GEGLU needs N % 256 == 0 (LL_ERR_UNSUPPORTED
+ * otherwise), runs on the FP8-operand kernel (AUTO and the two FP8
+ * variants; the others return LL_ERR_UNSUPPORTED from ll_forward), and
+ * stores the weights in its own row order: switching GEGLU on or off
+ * requires ll_set_weights again (a forward before that returns
+ * LL_ERR_NOT_READY).  LL_ERR_INVALID_ARG for an unknown epilogue. */
+int ll_set_epilogue(ll_handle h, int epilogue);
+
 /* No counterpart on the pages.  Select a kernel variant (LL_VARIANT_AUTO
  * picks by M).  LL_ERR_INVALID_ARG for an unknown variant. */
 int ll_set_variant(ll_handle h, int variant);
@@ -186,6 +208,30 @@ int ll_status(ll_handle h);
  * withhold_producer != 0 makes the main kernel's loader issue nothing, so
  * its consumers run into the timeout (used to test the timeout path). */
 int ll_set_debug(ll_handle h, int withhold_producer, uint64_t timeout_ns);
+
+/* LiteLinear README, "Usage": LiteLinear.from_dense, the SVD-based
+ * decomposition of a dense weight (and "Features": the factors A, B, Q_fp8,
+ * Q_scale_inv).  After the SVD, which the caller runs (A = U_r S_r and
+ * B = V_r^T rounded to bf16, as the MoDeGPT compressor keeps them), this
+ * call quantises the residual:
+ *
+ *   R[n, k] = W[n, k] - sum_j A[n, j] B[j, k]   (binary64, j in order)
+ *   scale   = max |R| / 448 rounded to binary32, per row ([N]) or over the
+ *             whole tensor ([1]) by scale_mode; 0 for an all-zero residual
+ *   Q[n, k] = e4m3fn code nearest to binary32(R[n, k] / scale) (ties to
+ *             even, saturating at 448); 0 where the scale is 0
+ *
+ * The pages do not state how the scale is chosen; this maps each row's (or
+ * the tensor's) largest residual to the largest e4m3fn value.  Device
+ * pointers: W bf16 [N, K], A bf16 [N, r] and B bf16 [r, K] (NULL when
+ * r == 0), Q uint8 [N, K], scale fp32 [N] or [1]; 2-byte alignment for
+ * the bf16 arrays, 4 for scale.  Asynchronous on `stream` (a per-tensor
+ * scale uses a stream-ordered allocation of N doubles).  Errors:
+ * LL_ERR_INVALID_ARG for bad sizes, mode or pointers, LL_ERR_UNSUPPORTED
+ * for K + r beyond 29,000 (the residual row is kept in shared memory),
+ * LL_ERR_OOM, LL_ERR_CUDA. */
+int ll_quantize_residual(const void *W, const void *A, const void *B, int N, int K, int r, int scale_mode, void *Q,
+                         float *scale, void *stream);
 
 /* The per-token e4m3fn quantisation of activations that the FP8-operand
  * variants apply before the residual product (the FP8-activation reading

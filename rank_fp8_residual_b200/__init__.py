@@ -38,6 +38,10 @@ LL_VARIANT_STREAM = 4
 LL_VARIANT_FP8_SPLIT = 5
 LL_VARIANT_FP8_ACT = 6
 
+LL_EPILOGUE_NONE = 0
+LL_EPILOGUE_GELU_TANH = 1
+LL_EPILOGUE_GEGLU_TANH = 2
+
 # Every symbol the header declares, with (restype, argtypes).
 _P = ctypes.c_void_p
 _SIGNATURES = {
@@ -47,6 +51,7 @@ _SIGNATURES = {
     "ll_forward_host": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, _P]),
     "ll_reserve": (ctypes.c_int, [_P, ctypes.c_int]),
     "ll_set_variant": (ctypes.c_int, [_P, ctypes.c_int]),
+    "ll_set_epilogue": (ctypes.c_int, [_P, ctypes.c_int]),
     "ll_status": (ctypes.c_int, [_P]),
     "ll_set_debug": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_uint64]),
     "ll_destroy": (None, [_P]),
@@ -58,6 +63,8 @@ _SIGNATURES = {
     "ll_kernel_name": (ctypes.c_char_p, [_P, ctypes.c_int]),
     "ll_forward_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, _P]),
+    "ll_quantize_residual": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            _P, _P, _P]),
     "ll_quantize_x": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P]),
     "ll_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                _P, _P, _P]),
@@ -147,6 +154,12 @@ def ll_set_variant(h: int, variant: int) -> None:
         raise LLError(rc, "ll_set_variant")
 
 
+def ll_set_epilogue(h: int, epilogue: int) -> None:
+    rc = _lib.ll_set_epilogue(h, int(epilogue))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_set_epilogue")
+
+
 def ll_status(h: int) -> int:
     return _lib.ll_status(h)
 
@@ -202,6 +215,37 @@ def ll_quantize_x(x, M: int, K: int, terms: int, e_out, hi, lo=None, stream=None
         raise LLError(rc, "ll_quantize_x")
 
 
+def ll_quantize_residual(W, A, B, N: int, K: int, r: int, scale_mode: int, Q, scale, stream=None) -> None:
+    """Residual codes and scale of the decomposition step (device buffers):
+    W bf16 [N, K], A bf16 [N, r], B bf16 [r, K] -> Q uint8 [N, K], scale
+    float32 [N] or [1]."""
+    rc = _lib.ll_quantize_residual(_addr(W), _addr(A), _addr(B), int(N), int(K), int(r), int(scale_mode), _addr(Q),
+                                   _addr(scale), _stream(stream))
+    if rc != LL_OK:
+        raise LLError(rc, "ll_quantize_residual")
+
+
+def from_dense(W, r: int, scale_mode: int = LL_SCALE_PER_ROW):
+    """Decompose a dense weight W (CUDA bf16 [N, K], nn.Linear layout) into
+    the layer's factors (LiteLinear README, "Usage": from_dense):
+    A = U_r S_r and B = V_r^T from torch's SVD (a library routine, run once
+    when a layer is built), rounded to bf16, and the residual's e4m3fn codes
+    and scale from ll_quantize_residual.  Returns (A, B, Q, scale)."""
+    import torch
+    N, K = W.shape
+    r = int(r)
+    if r > 0:
+        U, S, Vh = torch.linalg.svd(W.to(torch.float32), full_matrices=False)
+        A = (U[:, :r] * S[:r]).to(torch.bfloat16).contiguous()
+        B = Vh[:r].to(torch.bfloat16).contiguous()
+    else:
+        A = B = None
+    Q = torch.empty(N, K, dtype=torch.uint8, device=W.device)
+    scale = torch.empty(N if scale_mode == LL_SCALE_PER_ROW else 1, dtype=torch.float32, device=W.device)
+    ll_quantize_residual(W.contiguous(), A, B, N, K, r, scale_mode, Q, scale)
+    return A, B, Q, scale
+
+
 def ll_plan(N: int, K: int, r: int, M: int, num_sms: int, variant: int = 0):
     """(kernel variant, tokens per tile, down-projection K splits) that a
     forward of M tokens would use on an (N, K, r) layer with num_sms SMs.
@@ -222,18 +266,35 @@ class LiteLinearLayer:
     bias bf16 [N] or None.
     """
 
-    def __init__(self, N: int, K: int, r: int, scale_mode: int = LL_SCALE_PER_ROW):
+    def __init__(self, N: int, K: int, r: int, scale_mode: int = LL_SCALE_PER_ROW,
+                 epilogue: int = LL_EPILOGUE_NONE):
         self.N, self.K, self.r, self.scale_mode = N, K, r, scale_mode
         self.handle = ll_create(N, K, r, scale_mode)
+        self.epilogue = epilogue
+        if epilogue != LL_EPILOGUE_NONE:
+            ll_set_epilogue(self.handle, epilogue)
+
+    @property
+    def out_features(self) -> int:
+        return self.N // 2 if self.epilogue == LL_EPILOGUE_GEGLU_TANH else self.N
 
     def set_weights(self, A, B, Q, scale, bias=None):
         ll_set_weights(self.handle, A, B, Q, scale, bias)
+
+    @classmethod
+    def from_dense(cls, W, r: int, bias=None, scale_mode: int = LL_SCALE_PER_ROW):
+        """A layer from a dense CUDA bf16 weight [out, in] (see from_dense)."""
+        N, K = W.shape
+        A, B, Q, scale = from_dense(W, r, scale_mode)
+        layer = cls(N, K, r, scale_mode)
+        layer.set_weights(A, B, Q, scale, bias)
+        return layer
 
     def forward(self, x, out=None, stream=None):
         import torch
         M = x.shape[0]
         if out is None:
-            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+            out = torch.empty(M, self.out_features, dtype=torch.bfloat16, device=x.device)
         ll_forward(self.handle, x, out, M, stream)
         return out
 

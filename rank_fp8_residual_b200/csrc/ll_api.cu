@@ -20,6 +20,7 @@
 #include "ll_tc2.cuh"
 #include "ll_stream.cuh"
 #include "ll_f8.cuh"
+#include "ll_decompose.cuh"
 
 namespace {
 
@@ -102,6 +103,32 @@ bool is_device_ptr_on(const void* p, int dev) {
   return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
 }
 
+// Stored row of original output feature n.  With a GEGLU epilogue, tile t
+// of 256 stored rows holds the value features 128t .. 128t + 127 and then
+// their gate features N/2 + 128t .. (so both halves of an output feature
+// meet in one thread of the FP8-operand kernel's epilogue); otherwise the
+// identity.
+int original_row(int stored, int N, bool geglu) {
+  if (!geglu) return stored;
+  const int t = stored / 256, i = stored % 256;
+  return i < 128 ? 128 * t + i : N / 2 + 128 * t + (i - 128);
+}
+
+// Device-to-device copy of N rows of `width` bytes into the stored order.
+bool copy_rows(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width, int N, bool geglu) {
+  if (!geglu)
+    return cudaMemcpy2D(dst, dpitch, src, spitch, width, N, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  bool ok = true;
+  for (int t = 0; t < N / 256; ++t)
+    for (int half = 0; half < 2; ++half) {
+      const int src_row = half == 0 ? 128 * t : N / 2 + 128 * t;
+      ok &= cudaMemcpy2D(static_cast<char*>(dst) + (256 * t + 128 * half) * dpitch, dpitch,
+                         static_cast<const char*>(src) + src_row * spitch, spitch, width, 128,
+                         cudaMemcpyDeviceToDevice) == cudaSuccess;
+    }
+  return ok;
+}
+
 // Byte ranges [a, a + na) and [b, b + nb) intersect.
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   const char* pa = static_cast<const char*>(a);
@@ -122,6 +149,23 @@ struct TcChoice {
   int bt;  // tokens per fused-kernel tile
   int ks;  // K splits of the down-projection (1 when r == 0)
 };
+
+// TMA descriptors that depend on the call's x, y and M (and on the
+// workspace, whose growth clears them).
+struct CallMaps {
+  const void* c_x = nullptr;
+  void* c_yptr = nullptr;
+  int c_M = -1;
+  bool c_f8 = false;  // the FP8-operand maps are built
+  CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256;
+  CUtensorMap c_xs, c_this, c_tlos;     // streaming kernel: x and t boxes of Mt rows
+  CUtensorMap c_xbt, c_thibt, c_tlobt;  // fused single-CTA kernel: x and t boxes of bt rows
+  int c_bt = 0;
+  CUtensorMap c_x2p, c_thip, c_tlop;  // CTA-pair kernel: x and t boxes of bt2 / 2 rows
+  int c_bt2 = 0;
+  CUtensorMap c_xh, c_xl, c_thi32, c_tlo32, c_y64;  // FP8-operand kernel
+};
+constexpr int kMapCache = 8;  // descriptor sets kept per layer (e.g. the chunks of a host-buffer forward)
 
 struct ll_layer {
   int N = 0, K = 0, r = 0, r_pad = 0, klr = 64, scale_mode = 0;
@@ -154,8 +198,6 @@ struct ll_layer {
   size_t f8_cnt_n = 0;
   float* f8_part = nullptr;  // fp32 partial tiles, two slots per CTA pair
   CUtensorMap tm_q128, tm_ahi32, tm_alo32;     // set-time maps of the FP8-operand kernel
-  CUtensorMap c_xh, c_xl, c_thi32, c_tlo32, c_y64;  // per-call maps of the FP8-operand kernel
-  bool c_f8 = false;                           // the per-call FP8 maps are built
   mutable int f8_clusters = 0;                 // co-resident clusters of the FP8-operand kernel
   // host-buffer forward staging: device copies of x and y, and two copy
   // streams (host to device, device to host) that overlap the chunks' copies
@@ -168,24 +210,19 @@ struct ll_layer {
   // weight tensor maps
   CUtensorMap tm_q, tm_qf, tm_a, tm_ahi, tm_alo, tm_b;
   int b_box = 0;
-  // per-call cache
-  const void* c_x = nullptr;
-  void* c_yptr = nullptr;
-  int c_M = -1;
-  CUtensorMap c_x128, c_x256, c_y, c_thi128, c_tlo128, c_thi256, c_tlo256;
-  CUtensorMap c_xs, c_this, c_tlos;  // streaming kernel: x and t boxes of Mt rows
+  // per-call descriptors: the current set, and the last kMapCache sets built
+  CallMaps cm;
+  CallMaps cm_cache[kMapCache];
+  int cm_next = 0;
   CUtensorMap tm_q3;  // 3-D view of the (row-cleared) residual, 4 K chunks per box
   CUtensorMap tm_q3b2;  // the same view, 2 K chunks per box (fused single-CTA kernel)
-  CUtensorMap c_xbt, c_thibt, c_tlobt;  // fused single-CTA kernel: x and t boxes of bt rows
-  int c_bt = 0;
   mutable int tcp_M = -1;  // M of the cached joint plan (single-CTA kernel)
   mutable TcChoice tcp{};
   mutable int tcp2_M = -1;  // M of the cached joint plan (CTA-pair kernel)
   mutable TcChoice tcp2{};
-  CUtensorMap c_x2p, c_thip, c_tlop;  // CTA-pair kernel: x and t boxes of bt2 / 2 rows
-  int c_bt2 = 0;
   mutable int pair_clusters = 0;  // co-resident clusters of the CTA-pair kernel
   int variant = LL_VARIANT_AUTO;
+  int epilogue = LL_EPILOGUE_NONE;  // activation fused into the epilogue
   int withhold = 0;
   uint64_t timeout_ns = 2000000000ull;
   int last_launches = 0;
@@ -255,6 +292,12 @@ int set_smem_attrs_once() {
   return rc;
 }
 
+// Invalidates every descriptor set (the workspace they point into moved).
+void clear_call_maps(ll_layer* h) {
+  h->cm.c_M = -1;
+  for (CallMaps& c : h->cm_cache) c.c_M = -1;
+}
+
 // Grow the t workspace to hold `M` rows (stream-ordered).
 int ensure_workspace(ll_layer* h, int M, cudaStream_t st) {
   if (h->r_pad == 0) return LL_OK;
@@ -274,7 +317,7 @@ int ensure_workspace(ll_layer* h, int M, cudaStream_t st) {
     h->t_hi = th;
     h->t_lo = tl;
     h->ws_M = newM;
-    h->c_M = -1;  // maps over t must be rebuilt
+    clear_call_maps(h);  // maps over t must be rebuilt
   }
   return LL_OK;
 }
@@ -322,11 +365,17 @@ int ensure_f8_workspace(ll_layer* h, int M, cudaStream_t st) {
   h->f8_cnt = cnt;
   h->f8_cnt_n = ncnt;
   h->ws8_M = newM;
-  h->c_M = -1;  // maps over the codes must be rebuilt
+  clear_call_maps(h);  // maps over the codes must be rebuilt
   return LL_OK;
 }
 
 enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM, PATH_F8 };
+
+bool is_geglu(const ll_layer* h) { return h->epilogue == LL_EPILOGUE_GEGLU_TANH; }
+// Columns of y: N, or N / 2 when the epilogue is GEGLU.
+int out_features(const ll_layer* h) { return is_geglu(h) ? h->N / 2 : h->N; }
+// Activation code of the kernels' epilogues (epi_act).
+int act_code(const ll_layer* h) { return h->epilogue == LL_EPILOGUE_GELU_TANH ? 1 : 0; }
 
 // Where the two-term FP8-operand kernel beats the one-CTA exact-widening
 // kernel for M > 256.  Its split of x costs 2MK bytes each way against a
@@ -343,6 +392,9 @@ constexpr int kPairMaxM = 256;
 
 Path choose_path(const ll_layer* h, int M) {
   if (h->variant == LL_VARIANT_FP8_SPLIT || h->variant == LL_VARIANT_FP8_ACT) return PATH_F8;
+  // GEGLU pairs value and gate features inside a thread: the FP8-operand
+  // kernel holds a token's features in one thread; the others do not.
+  if (is_geglu(h) && h->variant == LL_VARIANT_AUTO) return PATH_F8;
   if (h->variant == LL_VARIANT_TC) return PATH_TC1;
   if (h->variant == LL_VARIANT_TC_PAIR) return PATH_TC2;
   if (h->variant == LL_VARIANT_SMALL) return PATH_SMALL;
@@ -529,89 +581,110 @@ cudaError_t launch_lrdown(const llk::LrDownParams& lpp, const LrPlan& lp, cudaSt
   return cudaLaunchKernelEx(&cfg, llk::ll_lrdown_kernel, lpp);
 }
 
+bool build_call_maps_uncached(ll_layer* h, const void* x, void* y, int M, bool f8);
+
+// The descriptor set of (x, y, M): the current one, a cached one, or a new
+// one (kept in the cache, oldest entry replaced).
 bool build_call_maps(ll_layer* h, const void* x, void* y, int M, bool f8) {
-  if (h->c_x == x && h->c_yptr == y && h->c_M == M && (!f8 || h->c_f8)) return true;
+  auto match = [&](const CallMaps& c) { return c.c_x == x && c.c_yptr == y && c.c_M == M && (!f8 || c.c_f8); };
+  if (match(h->cm)) return true;
+  for (const CallMaps& c : h->cm_cache)
+    if (match(c)) {
+      h->cm = c;
+      return true;
+    }
+  if (!build_call_maps_uncached(h, x, y, M, f8)) return false;
+  h->cm_cache[h->cm_next] = h->cm;
+  h->cm_next = (h->cm_next + 1) % kMapCache;
+  return true;
+}
+
+bool build_call_maps_uncached(ll_layer* h, const void* x, void* y, int M, bool f8) {
   using namespace llk;
   bool ok = true;
   if (f8) {
     constexpr CUtensorMapDataType kU8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    ok &= make_map(&h->c_xh, h->xh, kU8, M, h->K, h->K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&h->c_xl, h->xl, kU8, M, h->K, h->K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&h->c_y64, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    ok &= make_map(&h->cm.c_xh, h->xh, kU8, M, h->K, h->K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->cm.c_xl, h->xl, kU8, M, h->K, h->K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->cm.c_y64, y, kBF16, M, out_features(h), 2ull * out_features(h), 32, 32,
+                   CU_TENSOR_MAP_SWIZZLE_64B);
     if (h->r_pad > 0) {
-      ok &= make_map(&h->c_thi32, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
-      ok &= make_map(&h->c_tlo32, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+      ok &= make_map(&h->cm.c_thi32, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+      ok &= make_map(&h->cm.c_tlo32, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
     }
   }
-  h->c_f8 = f8;
-  ok &= make_map(&h->c_x128, x, kBF16, M, h->K, 2ull * h->K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&h->c_x256, x, kBF16, M, h->K, 2ull * h->K, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&h->c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  h->cm.c_f8 = f8;
+  ok &= make_map(&h->cm.c_x128, x, kBF16, M, h->K, 2ull * h->K, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&h->cm.c_x256, x, kBF16, M, h->K, 2ull * h->K, kBK, 256, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&h->cm.c_y, y, kBF16, M, h->N, 2ull * h->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (M > 128) {
     const int bt = tc_tile_tokens(h, M);
-    h->c_bt = bt;
-    ok &= make_map(&h->c_xbt, x, kBF16, M, h->K, 2ull * h->K, kBK, bt, CU_TENSOR_MAP_SWIZZLE_128B);
+    h->cm.c_bt = bt;
+    ok &= make_map(&h->cm.c_xbt, x, kBF16, M, h->K, 2ull * h->K, kBK, bt, CU_TENSOR_MAP_SWIZZLE_128B);
     if (h->r_pad > 0) {
       const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-      ok &= make_map(&h->c_thibt, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
-      ok &= make_map(&h->c_tlobt, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
+      ok &= make_map(&h->cm.c_thibt, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
+      ok &= make_map(&h->cm.c_tlobt, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, bt, sw);
     }
   }
   {
     // CTA-pair kernel maps (every M: any variant may be chosen later).
     const int bt2 = tc2_tile_tokens(h, M);
     const uint32_t hb = static_cast<uint32_t>(bt2 / 2);
-    h->c_bt2 = bt2;
+    h->cm.c_bt2 = bt2;
     if (h->K % 64 == 0)
-      ok &= make_map3(&h->c_x2p, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, hb, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map3(&h->cm.c_x2p, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, hb, 2, CU_TENSOR_MAP_SWIZZLE_128B);
     else
-      ok &= make_map(&h->c_x2p, x, kBF16, M, h->K, 2ull * h->K, kBK, hb, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&h->cm.c_x2p, x, kBF16, M, h->K, 2ull * h->K, kBK, hb, CU_TENSOR_MAP_SWIZZLE_128B);
     if (h->r_pad > 0) {
       const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-      ok &= make_map(&h->c_thip, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, hb, sw);
-      ok &= make_map(&h->c_tlop, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, hb, sw);
+      ok &= make_map(&h->cm.c_thip, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, hb, sw);
+      ok &= make_map(&h->cm.c_tlop, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, hb, sw);
     }
   }
   if (M <= kStreamMaxM) {
     const uint32_t Mt = static_cast<uint32_t>((M + 15) / 16 * 16);
     if (h->K % 64 == 0)
-      ok &= make_map3(&h->c_xs, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, Mt, 4, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map3(&h->cm.c_xs, x, kBF16, 64, M, h->K / 64, 2ull * h->K, 128, 64, Mt, 4, CU_TENSOR_MAP_SWIZZLE_128B);
     else
-      ok &= make_map(&h->c_xs, x, kBF16, M, h->K, 2ull * h->K, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&h->cm.c_xs, x, kBF16, M, h->K, 2ull * h->K, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
     if (h->r_pad > 0) {
-      ok &= make_map(&h->c_this, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
-      ok &= make_map(&h->c_tlos, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&h->cm.c_this, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&h->cm.c_tlos, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
     }
   }
   if (h->r_pad > 0) {
     const CUtensorMapSwizzle sw = h->klr == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    ok &= make_map(&h->c_thi128, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&h->c_tlo128, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&h->c_thi256, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
-    ok &= make_map(&h->c_tlo256, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
+    ok &= make_map(&h->cm.c_thi128, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->cm.c_tlo128, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&h->cm.c_thi256, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
+    ok &= make_map(&h->cm.c_tlo256, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, h->klr, 256, sw);
   }
   if (!ok) {
-    h->c_M = -1;
+    h->cm.c_M = -1;
     return false;
   }
-  h->c_x = x;
-  h->c_yptr = y;
-  h->c_M = M;
+  h->cm.c_x = x;
+  h->cm.c_yptr = y;
+  h->cm.c_M = M;
   return true;
 }
 
 // Data-parallel waves of the FP8-operand kernel before its stream-K tiles.
-// By default every tile is whole and taken from the counter (measured on
-// B200: the stream-K tail's partial sums and the pairs' uneven start times,
-// while the down-projection still holds SMs, cost more than the last
-// partial wave).  LL_FP8_STREAMK=1 in the environment spreads the last
-// partial wave (with the last whole wave when it is short) stream-K.
+// By default every tile is whole and taken from the counter.  Measured on
+// B200, spreading the last partial wave stream-K over all pairs does not
+// pay: the attention projection (120 tiles on 74 pairs) took 77 us against
+// 56 us whole, its split tiles' fp32 partials costing 4 to 13 us of memory
+// latency per pair in the epilogue.  LL_FP8_STREAMK=1 in the environment
+// turns the stream-K tail on (the last partial wave, merged with the whole
+// wave before it when it is shorter than half a wave), for measurements.
 int f8_dp_waves(int tiles, int clusters) {
   static const int sk = [] {
     const char* e = std::getenv("LL_FP8_STREAMK");
     return e && e[0] == '1' ? 1 : 0;
   }();
-  if (!sk) return (tiles + clusters - 1) / clusters;
+  const int whole = (tiles + clusters - 1) / clusters;
+  if (!sk) return whole;
   int D = tiles / clusters;
   const int S = tiles - D * clusters;
   if (S > 0 && D > 0 && 2 * S < clusters) --D;
@@ -653,6 +726,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   using namespace llk;
   h->last_launches = 0;
   const Path path = choose_path(h, M);
+  if (is_geglu(h) && path != PATH_F8) return LL_ERR_UNSUPPORTED;
   const LrPlan lp = plan_lowrank(h, M);
   int rc = ensure_workspace(h, M, st);
   if (rc != LL_OK) return rc;
@@ -690,7 +764,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
       h->b_box = lp.rc;
     }
     LrDownParams lpp;
-    lpp.tm_x = h->c_x128;
+    lpp.tm_x = h->cm.c_x128;
     lpp.tm_b = h->tm_b;
     lpp.t_hi = h->t_hi;
     lpp.t_lo = h->t_lo;
@@ -726,14 +800,14 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   cudaError_t err;
   if (path == PATH_F8) {
     F8Params fp;
-    fp.tm_xh = h->c_xh;
-    fp.tm_xl = h->c_xl;
+    fp.tm_xh = h->cm.c_xh;
+    fp.tm_xl = h->cm.c_xl;
     fp.tm_q = h->tm_q128;
     fp.tm_ahi = h->tm_ahi32;
     fp.tm_alo = h->tm_alo32;
-    fp.tm_thi = h->r_pad > 0 ? h->c_thi32 : h->c_xh;  // unused when r_pad == 0
-    fp.tm_tlo = h->r_pad > 0 ? h->c_tlo32 : h->c_xh;
-    fp.tm_y = h->c_y64;
+    fp.tm_thi = h->r_pad > 0 ? h->cm.c_thi32 : h->cm.c_xh;  // unused when r_pad == 0
+    fp.tm_tlo = h->r_pad > 0 ? h->cm.c_tlo32 : h->cm.c_xh;
+    fp.tm_y = h->cm.c_y64;
     fp.e_tok = h->e_tok;
     fp.scale = h->scale_eff;
     fp.bias = h->has_bias ? h->bias : nullptr;
@@ -749,12 +823,22 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     fp.n_ftiles = (h->N + 255) / 256;
     fp.lr_from_primary = overlap ? 1 : 0;
     fp.withhold = h->withhold;
+    fp.act = act_code(h);
+    fp.geglu = is_geglu(h) ? 1 : 0;
     fp.watch = watch;
     // Stream-K over (tile, 128-wide K step) units: one equal range per pair.
     const long long units = static_cast<long long>(fp.n_ttiles) * fp.n_ftiles * ((h->K + 127) / 128);
     const int clusters = static_cast<int>(std::max(1LL, std::min<long long>(f8_cluster_count(h), units)));
     fp.clusters = clusters;
-    fp.dp_waves = f8_dp_waves(fp.n_ttiles * fp.n_ftiles, clusters);
+    fp.dp_waves = is_geglu(h) ? (fp.n_ttiles * fp.n_ftiles + clusters - 1) / clusters
+                              : f8_dp_waves(fp.n_ttiles * fp.n_ftiles, clusters);
+    if (fp.dp_waves * clusters < fp.n_ttiles * fp.n_ftiles) {
+      // Stream-K splits the last wave evenly over all pairs, so they must
+      // all start together: no overlap with the down-projection, which
+      // would hold some SMs at the start.
+      cfg.numAttrs = 0;
+      fp.lr_from_primary = 0;
+    }
     cfg.gridDim = dim3(2 * clusters);
     cfg.blockDim = dim3(kF8Threads);
     cfg.dynamicSmemBytes = f8_smem_bytes();
@@ -763,11 +847,11 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   } else if (path == PATH_STREAM) {
     StreamParams sp;
     const bool dims3 = h->K % 64 == 0;
-    sp.tm_x = h->c_xs;
+    sp.tm_x = h->cm.c_xs;
     sp.tm_q = dims3 ? h->tm_q3 : h->tm_q;
     sp.tm_a = h->tm_a;
-    sp.tm_thi = h->c_this;
-    sp.tm_tlo = h->c_tlos;
+    sp.tm_thi = h->cm.c_this;
+    sp.tm_tlo = h->cm.c_tlos;
     sp.scale = h->scale;
     sp.bias = h->has_bias ? h->bias : nullptr;
     sp.y = static_cast<uint16_t*>(y);
@@ -780,6 +864,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     sp.dims3 = dims3 ? 1 : 0;
     sp.lr_from_primary = overlap ? 1 : 0;
     sp.withhold = h->withhold;
+    sp.act = act_code(h);
     sp.watch = watch;
     cfg.gridDim = dim3(stream_ctas(h));
     cfg.blockDim = dim3(kStThreads);
@@ -789,13 +874,13 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   } else if (path == PATH_TC2) {
     Tc2Params tp;
     tp.dims3 = h->K % 64 == 0 ? 1 : 0;
-    tp.tm_x = h->c_x2p;
+    tp.tm_x = h->cm.c_x2p;
     tp.tm_q = tp.dims3 ? h->tm_q3b2 : h->tm_qf;
     tp.tm_ahi = h->tm_ahi;
     tp.tm_alo = h->tm_alo;
-    tp.tm_thi = h->c_thip;
-    tp.tm_tlo = h->c_tlop;
-    tp.tm_y = h->c_y;
+    tp.tm_thi = h->cm.c_thip;
+    tp.tm_tlo = h->cm.c_tlop;
+    tp.tm_y = h->cm.c_y;
     tp.scale = h->scale_eff;
     tp.bias = h->has_bias ? h->bias : nullptr;
     tp.M = M;
@@ -803,7 +888,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     tp.K = h->K;
     tp.r_pad = h->r_pad;
     tp.klr = h->klr;
-    tp.bt = h->c_bt2;
+    tp.bt = h->cm.c_bt2;
     tp.n_fpairs = (h->N + 255) / 256;
     tp.n_ttiles = (M + tp.bt - 1) / tp.bt;
     tp.sched = h->sched;
@@ -811,6 +896,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     const int clusters = std::max(1, std::min(pair_cluster_count(h), tiles));
     tp.lr_from_primary = overlap ? 1 : 0;
     tp.withhold = h->withhold;
+    tp.act = act_code(h);
     tp.watch = watch;
     cfg.gridDim = dim3(2 * clusters);
     cfg.blockDim = dim3(kT2Threads);
@@ -820,15 +906,15 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   } else if (path == PATH_TC1) {
     TcParams tp;
     const bool large = M > 128;  // the per-call maps of bt rows exist for M > 128
-    tp.bt = large ? h->c_bt : 256;
-    tp.tm_x = large ? h->c_xbt : h->c_x256;
+    tp.bt = large ? h->cm.c_bt : 256;
+    tp.tm_x = large ? h->cm.c_xbt : h->cm.c_x256;
     tp.q3 = h->K % 64 == 0 ? 1 : 0;
     tp.tm_q = tp.q3 ? h->tm_q3b2 : h->tm_qf;
     tp.tm_ahi = h->tm_ahi;
     tp.tm_alo = h->tm_alo;
-    tp.tm_thi = large ? h->c_thibt : h->c_thi256;
-    tp.tm_tlo = large ? h->c_tlobt : h->c_tlo256;
-    tp.tm_y = h->c_y;
+    tp.tm_thi = large ? h->cm.c_thibt : h->cm.c_thi256;
+    tp.tm_tlo = large ? h->cm.c_tlobt : h->cm.c_tlo256;
+    tp.tm_y = h->cm.c_y;
     tp.scale = h->scale_eff;
     tp.bias = h->has_bias ? h->bias : nullptr;
     tp.sched = h->sched;
@@ -841,6 +927,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     tp.n_ttiles = (M + tp.bt - 1) / tp.bt;
     tp.lr_from_primary = overlap ? 1 : 0;
     tp.withhold = h->withhold;
+    tp.act = act_code(h);
     tp.watch = watch;
     const int tiles = tp.n_ftiles * tp.n_ttiles;
     cfg.gridDim = dim3(std::min(tiles, h->num_sms));
@@ -850,12 +937,12 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     h->names[launches] = "ll_tc_kernel";
   } else {
     MainParams mp;
-    mp.tm_x = h->c_x128;
+    mp.tm_x = h->cm.c_x128;
     mp.tm_q = h->tm_q;
     mp.tm_a = h->tm_a;
-    mp.tm_thi = h->c_thi128;
-    mp.tm_tlo = h->c_tlo128;
-    mp.tm_y = h->c_y;
+    mp.tm_thi = h->cm.c_thi128;
+    mp.tm_tlo = h->cm.c_tlo128;
+    mp.tm_y = h->cm.c_y;
     mp.scale = h->scale;
     mp.bias = h->has_bias ? h->bias : nullptr;
     mp.M = M;
@@ -866,6 +953,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     mp.n_ttiles = (M + 127) / 128;
     mp.lr_from_primary = overlap ? 1 : 0;
     mp.withhold = h->withhold;
+    mp.act = act_code(h);
     mp.watch = watch;
     const int tiles = mp.n_ftiles * mp.n_ttiles;
     cfg.gridDim = dim3(std::min(tiles, h->num_sms));
@@ -1024,7 +1112,7 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
   std::vector<float> full(N), eff(N);
   bool any_zero = false;
   for (int n = 0; n < N; ++n) {
-    full[n] = hs[h->scale_mode == LL_SCALE_PER_ROW ? n : 0];
+    full[n] = hs[h->scale_mode == LL_SCALE_PER_ROW ? original_row(n, N, is_geglu(h)) : 0];
     eff[n] = full[n] == 0.f ? 1.f : full[n];
     any_zero |= full[n] == 0.f;
   }
@@ -1042,11 +1130,11 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
   if (flag) return fail(LL_ERR_NAN_CODE);
   h->ready = false;
   bool ok = true;
-  ok &= cudaMemcpy(h->Q, Q, nq, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= copy_rows(h->Q, K, Q, K, K, N, is_geglu(h));
   ok &= cudaMemcpy(h->scale, full.data(), sizeof(float) * N, cudaMemcpyHostToDevice) == cudaSuccess;
   ok &= cudaMemcpy(h->scale_eff, eff.data(), sizeof(float) * N, cudaMemcpyHostToDevice) == cudaSuccess;
   if (bias) {
-    ok &= cudaMemcpy(h->bias, bias, sizeof(uint16_t) * N, cudaMemcpyDeviceToDevice) == cudaSuccess;
+    ok &= copy_rows(h->bias, sizeof(uint16_t), bias, sizeof(uint16_t), sizeof(uint16_t), N, is_geglu(h));
   } else {
     ok &= cudaMemset(h->bias, 0, sizeof(uint16_t) * N) == cudaSuccess;
   }
@@ -1085,8 +1173,7 @@ int ll_set_weights(ll_handle h, const void* A, const void* B, const void* Q, con
   if (rp > 0) {
     ok &= cudaMemset(h->A, 0, sizeof(uint16_t) * N * static_cast<size_t>(rp)) == cudaSuccess;
     ok &= cudaMemset(h->B, 0, sizeof(uint16_t) * static_cast<size_t>(rp) * K) == cudaSuccess;
-    ok &= cudaMemcpy2D(h->A, sizeof(uint16_t) * rp, A, sizeof(uint16_t) * r, sizeof(uint16_t) * r, N,
-                       cudaMemcpyDeviceToDevice) == cudaSuccess;
+    ok &= copy_rows(h->A, sizeof(uint16_t) * rp, A, sizeof(uint16_t) * r, sizeof(uint16_t) * r, N, is_geglu(h));
     ok &= cudaMemcpy(h->B, B, sizeof(uint16_t) * static_cast<size_t>(r) * K, cudaMemcpyDeviceToDevice) ==
           cudaSuccess;
     if (ok) {
@@ -1122,7 +1209,7 @@ int ll_forward(ll_handle h, const void* x, void* y, int M, void* stream) {
   if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return fail(LL_ERR_INVALID_ARG);
   const char* xb = static_cast<const char*>(x);
   const char* yb = static_cast<const char*>(y);
-  const size_t xs = static_cast<size_t>(M) * h->K * 2, ys = static_cast<size_t>(M) * h->N * 2;
+  const size_t xs = static_cast<size_t>(M) * h->K * 2, ys = static_cast<size_t>(M) * out_features(h) * 2;
   if (xb < yb + ys && yb < xb + xs) return fail(LL_ERR_INVALID_ARG);
   int rc = forward_device(h, x, y, M, static_cast<cudaStream_t>(stream));
   return rc == LL_OK ? LL_OK : fail(rc);
@@ -1135,7 +1222,7 @@ int ll_forward_host(ll_handle h, const void* x_host, void* y_host, int M, void* 
   if (!h->ready) return fail(LL_ERR_NOT_READY);
   if (M == 0) return LL_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t xrow = static_cast<size_t>(h->K) * 2, yrow = static_cast<size_t>(h->N) * 2;
+  const size_t xrow = static_cast<size_t>(h->K) * 2, yrow = static_cast<size_t>(out_features(h)) * 2;
   const size_t xs = static_cast<size_t>(M) * xrow, ys = static_cast<size_t>(M) * yrow;
   if (!h->cin) {
     bool ok = cudaStreamCreateWithFlags(&h->cin, cudaStreamNonBlocking) == cudaSuccess &&
@@ -1218,6 +1305,17 @@ int ll_reserve(ll_handle h, int max_M) {
     rc = LL_ERR_CUDA;
   }
   return rc == LL_OK ? LL_OK : fail(rc);
+}
+
+int ll_set_epilogue(ll_handle h, int epilogue) {
+  g_last_error = LL_OK;
+  if (!h || epilogue < LL_EPILOGUE_NONE || epilogue > LL_EPILOGUE_GEGLU_TANH) return fail(LL_ERR_INVALID_ARG);
+  if (epilogue == LL_EPILOGUE_GEGLU_TANH && h->N % 256 != 0) return fail(LL_ERR_UNSUPPORTED);
+  // The GEGLU row order is applied when the weights are copied in.
+  if ((epilogue == LL_EPILOGUE_GEGLU_TANH) != is_geglu(h)) h->ready = false;
+  h->epilogue = epilogue;
+  clear_call_maps(h);  // the width of y may change
+  return LL_OK;
 }
 
 int ll_set_variant(ll_handle h, int variant) {
@@ -1332,6 +1430,52 @@ int ll_kernel_times(ll_handle h, float* ms, int n) {
 const char* ll_kernel_name(ll_handle h, int i) {
   if (!h || i < 0 || i >= h->last_launches) return nullptr;
   return h->names[i];
+}
+
+int ll_quantize_residual(const void* W, const void* A, const void* B, int N, int K, int r, int scale_mode,
+                         void* Q, float* scale, void* stream) {
+  g_last_error = LL_OK;
+  if (N < 1 || K < 1 || r < 0 || (scale_mode != LL_SCALE_PER_TENSOR && scale_mode != LL_SCALE_PER_ROW))
+    return fail(LL_ERR_INVALID_ARG);
+  if (!W || !Q || !scale || (r > 0 && (!A || !B))) return fail(LL_ERR_INVALID_ARG);
+  if (!aligned(W, 2) || !aligned(scale, 4) || (r > 0 && (!aligned(A, 2) || !aligned(B, 2))))
+    return fail(LL_ERR_INVALID_ARG);
+  const size_t smem = llk::rq_smem_bytes(K, r);
+  if (smem > 227 * 1024) return fail(LL_ERR_UNSUPPORTED);
+  if (!is_device_ptr(W) || !is_device_ptr(Q) || !is_device_ptr(scale) ||
+      (r > 0 && (!is_device_ptr(A) || !is_device_ptr(B))))
+    return fail(LL_ERR_INVALID_ARG);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaFuncSetAttribute(llk::ll_residual_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(llk::ll_residual_tensor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_CUDA);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int blocks = std::max(1, std::min(N, sms * 4));
+  const auto* w = static_cast<const uint16_t*>(W);
+  const auto* a = r > 0 ? static_cast<const uint16_t*>(A) : nullptr;
+  const auto* b = r > 0 ? static_cast<const uint16_t*>(B) : nullptr;
+  auto* q = static_cast<uint8_t*>(Q);
+  if (scale_mode == LL_SCALE_PER_ROW) {
+    llk::ll_residual_rows_kernel<<<blocks, llk::kRqThreads, smem, st>>>(w, a, b, N, K, r, q, scale, nullptr);
+    if (cudaGetLastError() != cudaSuccess) return fail(LL_ERR_CUDA);
+    return LL_OK;
+  }
+  double* rowmax = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&rowmax), sizeof(double) * N, st) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LL_ERR_OOM);
+  }
+  llk::ll_residual_rows_kernel<<<blocks, llk::kRqThreads, smem, st>>>(w, a, b, N, K, r, q, scale, rowmax);
+  llk::ll_residual_tensor_kernel<<<blocks, llk::kRqThreads, smem, st>>>(w, a, b, N, K, r, q, scale, rowmax);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  cudaFreeAsync(rowmax, st);
+  if (!launched) return fail(LL_ERR_CUDA);
+  return LL_OK;
 }
 
 int ll_quantize_x(const void* x, int M, int K, int terms, int* e_out, void* hi, void* lo, void* stream) {
@@ -1534,6 +1678,7 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   mp.n_ttiles = (M + 127) / 128;
   mp.lr_from_primary = r_pad > 0 ? 1 : 0;
   mp.withhold = 0;
+  mp.act = 0;
   mp.watch = watch;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];

@@ -191,6 +191,8 @@ struct F8Params {
   int dp_waves;          // data-parallel waves of whole tiles before the stream-K tiles
   int lr_from_primary;   // 1: t' is written by the preceding kernel
   int withhold;          // debug: the producers issue nothing, so every consumer's wait runs out
+  int act;               // epilogue activation (epi_act)
+  int geglu;             // 1: y = h * gelu(g) over the halves of each tile's features (tm_y is [M, N/2])
   Watch watch;
 };
 
@@ -288,8 +290,22 @@ struct F8Sched {
   bool dp_done = false;
   int c, u, u_end;
   __device__ F8Sched(const F8Split& sp_, int c_) : sp(sp_), c(c_), u(sp_.begin(c_)), u_end(sp_.begin(c_ + 1)) {}
+  int wv = 0;  // whole tiles taken so far (static first waves)
   __device__ bool next(F8Seg& g, uint64_t* tile_full, uint64_t* tile_empty, int* tile_slot, const Watch& w,
                        int code, bool whole_warp) {
+    if (!dp_done && sp.S > 0) {
+      // With a stream-K tail the whole tiles are dealt out statically
+      // (pair c: c, C + c, ...), so every pair reaches its stream-K range
+      // after the same amount of work.
+      if (wv * sp.C + c < sp.DT) {
+        g.T = wv * sp.C + c;
+        g.k0 = 0;
+        g.k1 = sp.nS;
+        ++wv;
+        return true;
+      }
+      dp_done = true;
+    }
     if (!dp_done) {
       int T;
       if (tr.next(tile_full, tile_empty, tile_slot, w, code, whole_warp, T)) {
@@ -570,48 +586,97 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
         __threadfence();  // acquire: the other pairs' partials are visible
         if (lane == 0) *cnt = 0;
       }
-      for (int c = 0; c < 8; ++c) {
-        // Sum of the pairs' partials in K order, starting from zero (a
-        // fixed order, whichever pair arrives last); this pair's own term
-        // comes from TMEM.
+      if (p.geglu) {
+        // GEGLU: the set-time order puts the gate rows of output features
+        // fbase/2 + j (j < 128) at tile columns 128 + j, beside their value
+        // rows at columns j, so each thread has both for its token.  Whole
+        // tiles only (the host keeps the stream-K tail off).
+        for (int c = 0; c < 4; ++c) {
+          uint32_t vh[32], vg[32];
+          tmem_ld32x2_wait(acc + 32u * c, vh, acc + 128u + 32u * c, vg);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 h0 = prm[32 * c + 2 * i], h1 = prm[32 * c + 2 * i + 1];
+            const float2 g0 = prm[128 + 32 * c + 2 * i], g1 = prm[128 + 32 * c + 2 * i + 1];
+            const float o0 = fmaf(h0.x * sm, __uint_as_float(vh[2 * i]), h0.y) *
+                             gelu_tanh(fmaf(g0.x * sm, __uint_as_float(vg[2 * i]), g0.y));
+            const float o1 = fmaf(h1.x * sm, __uint_as_float(vh[2 * i + 1]), h1.y) *
+                             gelu_tanh(fmaf(g1.x * sm, __uint_as_float(vg[2 * i + 1]), g1.y));
+            w[i] = pack_bf16x2(o0, o1);
+          }
+          if (lane == 0) tma_store_wait_read<1>();
+          __syncwarp();
+          uint8_t* st = stg + eb * (32 * 64);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(st + lane * 64 + 16 * (j ^ sw)) =
+                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int fo = fbase / 2 + 32 * c;
+            if (trow < p.M && fo < p.N / 2) tma_store_2d(&p.tm_y, st, fo, trow);
+            tma_store_commit();
+          }
+          eb ^= 1;
+        }
+        release();
+        ++it;
+        continue;
+      }
+      // A split tile's other pairs' partials, four chunks (128 columns) of
+      // one pair per batch of loads, so a finish costs a few L2 round trips
+      // instead of one per chunk.
+      float4 pf[4][8];
+      for (int c0 = 0; c0 < 8; c0 += 4)
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = c0 + cc;
+        // Sum of the pairs' terms in K order, starting from zero (a fixed
+        // order, whichever pair arrives last); this pair's own term comes
+        // from TMEM.
         uint32_t v[32];
         tmem_ld32_wait(acc + 32u * c, v);
         float a[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) a[i] = split ? 0.f : __uint_as_float(v[i]);
-        for (int j = c_first; split && j <= c_last; j += 2) {
-          // two terms per batch of loads
-          const int j1 = j + 1 <= c_last ? j + 1 : -1;
-          float4 u0[8], u1[8];
-          const float4* s0 = j != cid ? reinterpret_cast<const float4*>(
-                                            p.part + (static_cast<size_t>(sp.slot(j, Ts)) * 2 + rank) * kF8PartFloats)
-                                      : nullptr;
-          const float4* s1 = j1 >= 0 && j1 != cid
-                                 ? reinterpret_cast<const float4*>(
-                                       p.part + (static_cast<size_t>(sp.slot(j1, Ts)) * 2 + rank) * kF8PartFloats)
-                                 : nullptr;
+        for (int j = c_first; split && j <= c_last; ++j) {
+          if (j == cid) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            u0[i] = s0 ? __ldcg(s0 + f8_part_at(row, c, i))
-                       : make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            u1[i] = s1 ? __ldcg(s1 + f8_part_at(row, c, i))
-                       : (j1 == cid ? make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f));
+            for (int i = 0; i < 32; ++i) a[i] += __uint_as_float(v[i]);
+            continue;
+          }
+          if (c_last - c_first == 1 && cc == 0) {
+            // two pairs: prefetch the other's next four chunks at once
+            const float4* s4 = reinterpret_cast<const float4*>(
+                p.part + (static_cast<size_t>(sp.slot(j, Ts)) * 2 + rank) * kF8PartFloats);
+#pragma unroll
+            for (int c2 = 0; c2 < 4; ++c2)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) pf[c2][i] = __ldcg(s4 + f8_part_at(row, c0 + c2, i));
+          }
+          float4 u[8];
+          if (c_last - c_first == 1) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = pf[cc][i];
+          } else {
+            const float4* s4 = reinterpret_cast<const float4*>(
+                p.part + (static_cast<size_t>(sp.slot(j, Ts)) * 2 + rank) * kF8PartFloats);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = __ldcg(s4 + f8_part_at(row, c, i));
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            a[4 * i] += u0[i].x; a[4 * i + 1] += u0[i].y; a[4 * i + 2] += u0[i].z; a[4 * i + 3] += u0[i].w;
-            if (j1 < 0) continue;
-            a[4 * i] += u1[i].x; a[4 * i + 1] += u1[i].y; a[4 * i + 2] += u1[i].z; a[4 * i + 3] += u1[i].w;
+            a[4 * i] += u[i].x; a[4 * i + 1] += u[i].y; a[4 * i + 2] += u[i].z; a[4 * i + 3] += u[i].w;
           }
         }
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 p0 = prm[32 * c + 2 * i], p1 = prm[32 * c + 2 * i + 1];  // broadcast reads
-          w[i] = pack_bf16x2(fmaf(p0.x * sm, a[2 * i], p0.y), fmaf(p1.x * sm, a[2 * i + 1], p1.y));
+          w[i] = pack_bf16x2(epi_act(fmaf(p0.x * sm, a[2 * i], p0.y), p.act),
+                             epi_act(fmaf(p1.x * sm, a[2 * i + 1], p1.y), p.act));
         }
         if (lane == 0) tma_store_wait_read<1>();
         __syncwarp();
@@ -646,7 +711,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
       uint32_t tph = 0;
       for (;;) {
         if (!mbar_wait_cl(&tile_empty[ti], tph ^ 1, p.watch, kErrTimeoutProducer)) break;
-        const int got = dp_tiles > 0 ? atomicAdd(&p.sched[0], 1) : dp_tiles;
+        // (no dynamic tiles when a stream-K tail deals them out statically)
+        const int got = dp_tiles > 0 && sp.S == 0 ? atomicAdd(&p.sched[0], 1) : dp_tiles;
         const int T = got < dp_tiles ? got : -1;
         *reinterpret_cast<volatile int*>(&tile_slot[ti]) = T;
         st_shared_cluster_u32(peer_slot + 4u * ti, static_cast<uint32_t>(T));

@@ -326,6 +326,7 @@ struct MainParams {
   int n_ftiles, n_ttiles;
   int lr_from_primary;  // 1: t is produced by the preceding kernel (wait on it)
   int withhold;         // debug: the TMA producer issues nothing
+  int act;              // epilogue activation (epi_act)
   Watch watch;
 };
 
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kMainThreads, 1) ll_main_kernel(const __grid_c
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float v = fmaf(s, __uint_as_float(aq[i]), __uint_as_float(al[i]) + b);
-          st[i * 32 + lane] = to_bf16_bits(v);
+          st[i * 32 + lane] = to_bf16_bits(epi_act(v, p.act));
         }
         fence_proxy_async_smem();
         __syncwarp();

@@ -63,6 +63,7 @@ struct TcParams {
   int q3;                // 1: one 3-D Q load per stage; 0: two 2-D loads
   int lr_from_primary;
   int withhold;
+  int act;               // epilogue activation (epi_act)
   Watch watch;
 };
 
@@ -441,7 +442,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
         __syncwarp();
         uint16_t* st = stage + eb * (32 * 32);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) st[i * 32 + lane] = to_bf16_bits(fmaf(s, __uint_as_float(v[i]), b));
+        for (int i = 0; i < 32; ++i) st[i * 32 + lane] = to_bf16_bits(epi_act(fmaf(s, __uint_as_float(v[i]), b), p.act));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

@@ -482,6 +482,15 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t v, uint32_t& lo, uint3
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(two120));
 }
 
+// Activation of the fused epilogue: 0 none, 1 GELU in its tanh form,
+// gelu(v) = v / 2 * (1 + tanh(sqrt(2 / pi) * (v + 0.044715 v^3))) (the
+// published tanh approximation of GELU, which the LTX feed-forward uses).
+__device__ __forceinline__ float gelu_tanh(float v) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
+  return 0.5f * v * (1.f + tanhf(u));
+}
+__device__ __forceinline__ float epi_act(float v, int act) { return act == 1 ? gelu_tanh(v) : v; }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

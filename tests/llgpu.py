@@ -14,10 +14,12 @@ import rank_fp8_residual_b200 as ll
 class DeviceLayer:
     """Library handle with the layer's factors uploaded."""
 
-    def __init__(self, inp, variant=ll.LL_VARIANT_AUTO):
+    def __init__(self, inp, variant=ll.LL_VARIANT_AUTO, epilogue=ll.LL_EPILOGUE_NONE):
         self.inp = inp
         self.h = ll.ll_create(inp.N, inp.K, inp.r, inp.scale_mode)
         ll.ll_set_variant(self.h, variant)
+        ll.ll_set_epilogue(self.h, epilogue)
+        self.n_out = inp.N // 2 if epilogue == ll.LL_EPILOGUE_GEGLU_TANH else inp.N
         dev = torch.device("cuda")
         self.A = inp.A.to(dev) if inp.A is not None else None
         self.B = inp.B.to(dev) if inp.B is not None else None
@@ -28,7 +30,7 @@ class DeviceLayer:
 
     def forward(self, x_cpu, stream=None):
         x = x_cpu.to("cuda")
-        y = torch.empty(x.shape[0], self.inp.N, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(x.shape[0], self.n_out, dtype=torch.bfloat16, device="cuda")
         ll.ll_forward(self.h, x, y, x.shape[0], stream)
         torch.cuda.synchronize()
         st = ll.ll_status(self.h)
@@ -39,8 +41,8 @@ class DeviceLayer:
         ll.ll_destroy(self.h)
 
 
-def run(inp, variant=ll.LL_VARIANT_AUTO):
-    d = DeviceLayer(inp, variant)
+def run(inp, variant=ll.LL_VARIANT_AUTO, epilogue=ll.LL_EPILOGUE_NONE):
+    d = DeviceLayer(inp, variant, epilogue)
     try:
         return d.forward(inp.x).cpu()
     finally:
