@@ -265,29 +265,43 @@ void free_layer_mem(ll_layer* h) {
   cudaFree(h->f8_part);
 }
 
+// The epilogue activation is a template parameter of each kernel (see
+// epi_act): one instantiation per activation code.
+using MainFn = void (*)(llk::MainParams);
+using TcFn = void (*)(llk::TcParams);
+using Tc2Fn = void (*)(llk::Tc2Params);
+using StreamFn = void (*)(llk::StreamParams);
+using F8Fn = void (*)(llk::F8Params);
+MainFn kernel_main(int act) { return act == llk::kActGelu ? llk::ll_main_kernel<llk::kActGelu> : llk::ll_main_kernel<llk::kActNone>; }
+TcFn kernel_tc(int act) { return act == llk::kActGelu ? llk::ll_tc_kernel<llk::kActGelu> : llk::ll_tc_kernel<llk::kActNone>; }
+Tc2Fn kernel_tc2(int act) { return act == llk::kActGelu ? llk::ll_tc2_kernel<llk::kActGelu> : llk::ll_tc2_kernel<llk::kActNone>; }
+StreamFn kernel_stream(int act) {
+  return act == llk::kActGelu ? llk::ll_stream_kernel<llk::kActGelu> : llk::ll_stream_kernel<llk::kActNone>;
+}
+F8Fn kernel_f8(int act) {
+  return act == llk::kActGeglu  ? llk::ll_f8_kernel<llk::kActGeglu>
+         : act == llk::kActGelu ? llk::ll_f8_kernel<llk::kActGelu>
+                                : llk::ll_f8_kernel<llk::kActNone>;
+}
+
 int set_smem_attrs_once() {
   static int rc = -1;
   static std::once_flag once;
   std::call_once(once, [] {
     rc = 0;
-    if (cudaFuncSetAttribute(llk::ll_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             llk::main_smem_bytes()) != cudaSuccess)
-      rc = 1;
-    if (cudaFuncSetAttribute(llk::ll_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             llk::tc_smem_bytes()) != cudaSuccess)
-      rc = 1;
-    if (cudaFuncSetAttribute(llk::ll_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             llk::tc2_smem_bytes()) != cudaSuccess)
-      rc = 1;
-    if (cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             llk::lr_smem_bytes(256)) != cudaSuccess)
-      rc = 1;
-    if (cudaFuncSetAttribute(llk::ll_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             llk::st_smem_max()) != cudaSuccess)
-      rc = 1;
-    if (cudaFuncSetAttribute(llk::ll_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             llk::f8_smem_bytes()) != cudaSuccess)
-      rc = 1;
+    auto smem = [](auto f, size_t bytes) {
+      if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+          cudaSuccess)
+        rc = 1;
+    };
+    for (int a = 0; a < 2; ++a) {
+      smem(kernel_main(a), llk::main_smem_bytes());
+      smem(kernel_tc(a), llk::tc_smem_bytes());
+      smem(kernel_tc2(a), llk::tc2_smem_bytes());
+      smem(kernel_stream(a), llk::st_smem_max());
+    }
+    for (int a = 0; a < 3; ++a) smem(kernel_f8(a), llk::f8_smem_bytes());
+    smem(llk::ll_lrdown_kernel, llk::lr_smem_bytes(256));
   });
   return rc;
 }
@@ -375,7 +389,11 @@ bool is_geglu(const ll_layer* h) { return h->epilogue == LL_EPILOGUE_GEGLU_TANH;
 // Columns of y: N, or N / 2 when the epilogue is GEGLU.
 int out_features(const ll_layer* h) { return is_geglu(h) ? h->N / 2 : h->N; }
 // Activation code of the kernels' epilogues (epi_act).
-int act_code(const ll_layer* h) { return h->epilogue == LL_EPILOGUE_GELU_TANH ? 1 : 0; }
+int act_code(const ll_layer* h) {
+  return h->epilogue == LL_EPILOGUE_GELU_TANH    ? llk::kActGelu
+         : h->epilogue == LL_EPILOGUE_GEGLU_TANH ? llk::kActGeglu
+                                                 : llk::kActNone;
+}
 
 // Where the two-term FP8-operand kernel beats the one-CTA exact-widening
 // kernel for M > 256.  Its split of x costs 2MK bytes each way against a
@@ -699,7 +717,7 @@ int f8_cluster_count(const ll_layer* h) {
   cfg.blockDim = dim3(llk::kF8Threads);
   cfg.dynamicSmemBytes = llk::f8_smem_bytes();
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, llk::ll_f8_kernel, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, kernel_f8(llk::kActNone), &cfg) != cudaSuccess || n <= 0) {
     cudaGetLastError();
     n = h->num_sms / 2;
   }
@@ -714,7 +732,7 @@ int pair_cluster_count(const ll_layer* h) {
   cfg.blockDim = dim3(llk::kT2Threads);
   cfg.dynamicSmemBytes = llk::tc2_smem_bytes();
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, llk::ll_tc2_kernel, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, kernel_tc2(llk::kActNone), &cfg) != cudaSuccess || n <= 0) {
     cudaGetLastError();
     n = h->num_sms / 2;
   }
@@ -823,8 +841,6 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     fp.n_ftiles = (h->N + 255) / 256;
     fp.lr_from_primary = overlap ? 1 : 0;
     fp.withhold = h->withhold;
-    fp.act = act_code(h);
-    fp.geglu = is_geglu(h) ? 1 : 0;
     fp.watch = watch;
     // Stream-K over (tile, 128-wide K step) units: one equal range per pair.
     const long long units = static_cast<long long>(fp.n_ttiles) * fp.n_ftiles * ((h->K + 127) / 128);
@@ -842,7 +858,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     cfg.gridDim = dim3(2 * clusters);
     cfg.blockDim = dim3(kF8Threads);
     cfg.dynamicSmemBytes = f8_smem_bytes();
-    err = cudaLaunchKernelEx(&cfg, ll_f8_kernel, fp);
+    err = cudaLaunchKernelEx(&cfg, kernel_f8(act_code(h)), fp);
     h->names[launches] = "ll_f8_kernel";
   } else if (path == PATH_STREAM) {
     StreamParams sp;
@@ -864,12 +880,11 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     sp.dims3 = dims3 ? 1 : 0;
     sp.lr_from_primary = overlap ? 1 : 0;
     sp.withhold = h->withhold;
-    sp.act = act_code(h);
     sp.watch = watch;
     cfg.gridDim = dim3(stream_ctas(h));
     cfg.blockDim = dim3(kStThreads);
     cfg.dynamicSmemBytes = st_smem_bytes(sp.Mt);
-    err = cudaLaunchKernelEx(&cfg, ll_stream_kernel, sp);
+    err = cudaLaunchKernelEx(&cfg, kernel_stream(act_code(h)), sp);
     h->names[launches] = "ll_stream_kernel";
   } else if (path == PATH_TC2) {
     Tc2Params tp;
@@ -896,12 +911,11 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     const int clusters = std::max(1, std::min(pair_cluster_count(h), tiles));
     tp.lr_from_primary = overlap ? 1 : 0;
     tp.withhold = h->withhold;
-    tp.act = act_code(h);
     tp.watch = watch;
     cfg.gridDim = dim3(2 * clusters);
     cfg.blockDim = dim3(kT2Threads);
     cfg.dynamicSmemBytes = tc2_smem_bytes();
-    err = cudaLaunchKernelEx(&cfg, ll_tc2_kernel, tp);
+    err = cudaLaunchKernelEx(&cfg, kernel_tc2(act_code(h)), tp);
     h->names[launches] = "ll_tc2_kernel";
   } else if (path == PATH_TC1) {
     TcParams tp;
@@ -927,13 +941,12 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     tp.n_ttiles = (M + tp.bt - 1) / tp.bt;
     tp.lr_from_primary = overlap ? 1 : 0;
     tp.withhold = h->withhold;
-    tp.act = act_code(h);
     tp.watch = watch;
     const int tiles = tp.n_ftiles * tp.n_ttiles;
     cfg.gridDim = dim3(std::min(tiles, h->num_sms));
     cfg.blockDim = dim3(kTcThreads);
     cfg.dynamicSmemBytes = tc_smem_bytes();
-    err = cudaLaunchKernelEx(&cfg, ll_tc_kernel, tp);
+    err = cudaLaunchKernelEx(&cfg, kernel_tc(act_code(h)), tp);
     h->names[launches] = "ll_tc_kernel";
   } else {
     MainParams mp;
@@ -953,13 +966,12 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     mp.n_ttiles = (M + 127) / 128;
     mp.lr_from_primary = overlap ? 1 : 0;
     mp.withhold = h->withhold;
-    mp.act = act_code(h);
     mp.watch = watch;
     const int tiles = mp.n_ftiles * mp.n_ttiles;
     cfg.gridDim = dim3(std::min(tiles, h->num_sms));
     cfg.blockDim = dim3(kMainThreads);
     cfg.dynamicSmemBytes = main_smem_bytes();
-    err = cudaLaunchKernelEx(&cfg, ll_main_kernel, mp);
+    err = cudaLaunchKernelEx(&cfg, kernel_main(act_code(h)), mp);
     h->names[launches] = "ll_main_kernel";
   }
   if (err != cudaSuccess) {
@@ -1252,6 +1264,10 @@ int ll_forward_host(ll_handle h, const void* x_host, void* y_host, int M, void* 
   // the same time (the two copy directions on their own streams).  The
   // caller's stream waits for the last copy out, so synchronising it once
   // still covers the whole call.
+  // Up to four chunks: the copies are the bound (tens of GB/s against the
+  // forward's TB/s).  Eight chunks measured slower than four on the
+  // attention projection (each copy and each forward has a fixed cost);
+  // below 512 tokens one chunk (each chunk reads the weights again).
   const int n_chunks = M >= 2048 ? 4 : (M >= 512 ? 2 : 1);
   const int rows = (M + n_chunks * 256 - 1) / (n_chunks * 256) * 256;
   cudaEvent_t* ev_in = h->hev + 1;
@@ -1547,7 +1563,7 @@ NoAllocDevice* noalloc_setup(int dev, int* rc) {
     int sms = 0;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0 ||
-        cudaFuncSetAttribute(llk::ll_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(kernel_main(llk::kActNone), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::main_smem_bytes()) != cudaSuccess ||
         cudaFuncSetAttribute(llk::ll_lrdown_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              llk::lr_smem_bytes(256)) != cudaSuccess) {
@@ -1678,7 +1694,6 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   mp.n_ttiles = (M + 127) / 128;
   mp.lr_from_primary = r_pad > 0 ? 1 : 0;
   mp.withhold = 0;
-  mp.act = 0;
   mp.watch = watch;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -1690,7 +1705,7 @@ int forward_noalloc(const void* x, const void* A, const void* B, const void* Q, 
   cfg.gridDim = dim3(std::min(mp.n_ftiles * mp.n_ttiles, d->num_sms));
   cfg.blockDim = dim3(kMainThreads);
   cfg.dynamicSmemBytes = main_smem_bytes();
-  if (cudaLaunchKernelEx(&cfg, ll_main_kernel, mp) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel_main(llk::kActNone), mp) != cudaSuccess) {
     cudaGetLastError();
     return LL_ERR_CUDA;
   }

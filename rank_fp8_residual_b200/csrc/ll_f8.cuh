@@ -191,8 +191,6 @@ struct F8Params {
   int dp_waves;          // data-parallel waves of whole tiles before the stream-K tiles
   int lr_from_primary;   // 1: t' is written by the preceding kernel
   int withhold;          // debug: the producers issue nothing, so every consumer's wait runs out
-  int act;               // epilogue activation (epi_act)
-  int geglu;             // 1: y = h * gelu(g) over the halves of each tile's features (tm_y is [M, N/2])
   Watch watch;
 };
 
@@ -204,6 +202,11 @@ constexpr int kF8EpiWarps = 4;
 constexpr int kF8SchedWarp = 2 + kF8EpiWarps;
 constexpr int kF8Threads = 32 * (kF8SchedWarp + 1);
 constexpr int kF8TileRing = 2;
+// The leader's producer asks for the next tile this many K steps before
+// the end of its current one, so a pair claims a tile only when it is about
+// to load it: pairs that start late (their SMs still held by the kernels
+// before) or run slow take fewer tiles instead of finding them claimed.
+constexpr int kF8ReqAhead = 3;
 constexpr int kF8EpiWarp = 2 * 32 * 64 + 256 * 8;  // per epilogue warp: two 32 x 32 bf16 staging buffers,
                                                      // then the tile's 256 (scale, bias) pairs
 constexpr int kF8Epi = kF8EpiWarps * kF8EpiWarp;
@@ -264,6 +267,7 @@ struct F8Split {
 };
 struct F8Seg {
   int T, k0, k1;
+  bool dyn;  // a whole tile taken from the scheduler's ring
 };
 // This CTA's view of the tile ring filled by the leader's scheduler.
 struct F8TileRing {
@@ -301,6 +305,7 @@ struct F8Sched {
         g.T = wv * sp.C + c;
         g.k0 = 0;
         g.k1 = sp.nS;
+        g.dyn = false;
         ++wv;
         return true;
       }
@@ -312,6 +317,7 @@ struct F8Sched {
         g.T = T;
         g.k0 = 0;
         g.k1 = sp.nS;
+        g.dyn = true;
         return true;
       }
       dp_done = true;
@@ -321,6 +327,7 @@ struct F8Sched {
     g.T = sp.DT + Ts;
     g.k0 = u - Ts * sp.nS;
     g.k1 = min(sp.nS, g.k0 + (u_end - u));
+    g.dyn = false;
     u += g.k1 - g.k0;
     return true;
   }
@@ -332,6 +339,9 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   return v;
 }
 
+// kAct: kActNone, kActGelu, or kActGeglu (y = h * gelu(g) over the halves of
+// each tile's features; tm_y is then [M, N/2]).
+template <int kAct>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
     ll_f8_kernel(const __grid_constant__ F8Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -345,7 +355,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
   uint64_t* tile_full = tempty + 2;
   uint64_t* tile_empty = tile_full + kF8TileRing;
   uint64_t* drain = tile_empty + kF8TileRing;
-  int* tile_slot = reinterpret_cast<int*>(drain + 1);
+  uint64_t* tile_req = drain + 1;  // leader: its producer wants the next tile
+  int* tile_slot = reinterpret_cast<int*>(tile_req + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_slot + kF8TileRing);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -374,6 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
       mbar_init(&tile_empty[s], 1 + kF8EpiWarps + (leader ? 2 : 0));
     }
     mbar_init(drain, 1);
+    mbar_init(tile_req, 1);
     fence_mbar_init();
     tma_prefetch_desc(&p.tm_xh);
     if (terms == 2) tma_prefetch_desc(&p.tm_xl);
@@ -419,6 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
           if (terms == 2) tma_load_2d_pair(dst + kF8Tile, &p.tm_xl, bar, s * 128, t0);
           tma_load_2d_pair(dst + terms * kF8Tile, &p.tm_q, bar, s * 128, f0);
           issued = true;
+          if (leader && g.dyn && s == max(g.k0, g.k1 - kF8ReqAhead)) mbar_arrive(tile_req);
           if (++slot == ns) { slot = 0; ph ^= 1; }
         }
         if (g.k0 != 0) continue;  // the low-rank term goes with a tile's first K steps
@@ -586,7 +599,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
         __threadfence();  // acquire: the other pairs' partials are visible
         if (lane == 0) *cnt = 0;
       }
-      if (p.geglu) {
+      if constexpr (kAct == kActGeglu) {
         // GEGLU: the set-time order puts the gate rows of output features
         // fbase/2 + j (j < 128) at tile columns 128 + j, beside their value
         // rows at columns j, so each thread has both for its token.  Whole
@@ -623,78 +636,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
         }
         release();
         ++it;
-        continue;
+      } else {
+        // A split tile's other pairs' partials, four chunks (128 columns) of
+        // one pair per batch of loads, so a finish costs a few L2 round trips
+        // instead of one per chunk.
+        float4 pf[4][8];
+        for (int c0 = 0; c0 < 8; c0 += 4)
+  #pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = c0 + cc;
+          // Sum of the pairs' terms in K order, starting from zero (a fixed
+          // order, whichever pair arrives last); this pair's own term comes
+          // from TMEM.
+          uint32_t v[32];
+          tmem_ld32_wait(acc + 32u * c, v);
+          float a[32];
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = split ? 0.f : __uint_as_float(v[i]);
+          for (int j = c_first; split && j <= c_last; ++j) {
+            if (j == cid) {
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) a[i] += __uint_as_float(v[i]);
+              continue;
+            }
+            if (c_last - c_first == 1 && cc == 0) {
+              // two pairs: prefetch the other's next four chunks at once
+              const float4* s4 = reinterpret_cast<const float4*>(
+                  p.part + (static_cast<size_t>(sp.slot(j, Ts)) * 2 + rank) * kF8PartFloats);
+  #pragma unroll
+              for (int c2 = 0; c2 < 4; ++c2)
+  #pragma unroll
+                for (int i = 0; i < 8; ++i) pf[c2][i] = __ldcg(s4 + f8_part_at(row, c0 + c2, i));
+            }
+            float4 u[8];
+            if (c_last - c_first == 1) {
+  #pragma unroll
+              for (int i = 0; i < 8; ++i) u[i] = pf[cc][i];
+            } else {
+              const float4* s4 = reinterpret_cast<const float4*>(
+                  p.part + (static_cast<size_t>(sp.slot(j, Ts)) * 2 + rank) * kF8PartFloats);
+  #pragma unroll
+              for (int i = 0; i < 8; ++i) u[i] = __ldcg(s4 + f8_part_at(row, c, i));
+            }
+  #pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              a[4 * i] += u[i].x; a[4 * i + 1] += u[i].y; a[4 * i + 2] += u[i].z; a[4 * i + 3] += u[i].w;
+            }
+          }
+          uint32_t w[16];
+  #pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 p0 = prm[32 * c + 2 * i], p1 = prm[32 * c + 2 * i + 1];  // broadcast reads
+            w[i] = pack_bf16x2(epi_act<kAct>(fmaf(p0.x * sm, a[2 * i], p0.y)),
+                               epi_act<kAct>(fmaf(p1.x * sm, a[2 * i + 1], p1.y)));
+          }
+          if (lane == 0) tma_store_wait_read<1>();
+          __syncwarp();
+          uint8_t* st = stg + eb * (32 * 64);
+  #pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(st + lane * 64 + 16 * (j ^ sw)) =
+                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (trow < p.M && fbase + 32 * c < p.N) tma_store_2d(&p.tm_y, st, fbase + 32 * c, trow);
+            tma_store_commit();
+          }
+          eb ^= 1;
+        }
+        release();
+        ++it;
       }
-      // A split tile's other pairs' partials, four chunks (128 columns) of
-      // one pair per batch of loads, so a finish costs a few L2 round trips
-      // instead of one per chunk.
-      float4 pf[4][8];
-      for (int c0 = 0; c0 < 8; c0 += 4)
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = c0 + cc;
-        // Sum of the pairs' terms in K order, starting from zero (a fixed
-        // order, whichever pair arrives last); this pair's own term comes
-        // from TMEM.
-        uint32_t v[32];
-        tmem_ld32_wait(acc + 32u * c, v);
-        float a[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) a[i] = split ? 0.f : __uint_as_float(v[i]);
-        for (int j = c_first; split && j <= c_last; ++j) {
-          if (j == cid) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) a[i] += __uint_as_float(v[i]);
-            continue;
-          }
-          if (c_last - c_first == 1 && cc == 0) {
-            // two pairs: prefetch the other's next four chunks at once
-            const float4* s4 = reinterpret_cast<const float4*>(
-                p.part + (static_cast<size_t>(sp.slot(j, Ts)) * 2 + rank) * kF8PartFloats);
-#pragma unroll
-            for (int c2 = 0; c2 < 4; ++c2)
-#pragma unroll
-              for (int i = 0; i < 8; ++i) pf[c2][i] = __ldcg(s4 + f8_part_at(row, c0 + c2, i));
-          }
-          float4 u[8];
-          if (c_last - c_first == 1) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = pf[cc][i];
-          } else {
-            const float4* s4 = reinterpret_cast<const float4*>(
-                p.part + (static_cast<size_t>(sp.slot(j, Ts)) * 2 + rank) * kF8PartFloats);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = __ldcg(s4 + f8_part_at(row, c, i));
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            a[4 * i] += u[i].x; a[4 * i + 1] += u[i].y; a[4 * i + 2] += u[i].z; a[4 * i + 3] += u[i].w;
-          }
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 p0 = prm[32 * c + 2 * i], p1 = prm[32 * c + 2 * i + 1];  // broadcast reads
-          w[i] = pack_bf16x2(epi_act(fmaf(p0.x * sm, a[2 * i], p0.y), p.act),
-                             epi_act(fmaf(p1.x * sm, a[2 * i + 1], p1.y), p.act));
-        }
-        if (lane == 0) tma_store_wait_read<1>();
-        __syncwarp();
-        uint8_t* st = stg + eb * (32 * 64);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(st + lane * 64 + 16 * (j ^ sw)) =
-              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (trow < p.M && fbase + 32 * c < p.N) tma_store_2d(&p.tm_y, st, fbase + 32 * c, trow);
-          tma_store_commit();
-        }
-        eb ^= 1;
-      }
-      release();
-      ++it;
     }
     if (lane == 0) tma_store_wait<0>();
   } else if (lane == 0) {
@@ -708,9 +721,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
       const uint32_t peer_slot = mapa_shared(smem_u32(&tile_slot[0]), 1);
       const uint32_t peer_full = mapa_shared(smem_u32(&tile_full[0]), 1);
       int ti = 0;
-      uint32_t tph = 0;
-      for (;;) {
+      uint32_t tph = 0, rph = 0;
+      for (bool first = true;; first = false) {
         if (!mbar_wait_cl(&tile_empty[ti], tph ^ 1, p.watch, kErrTimeoutProducer)) break;
+        // every claim after the first waits for the producer's request
+        if (!first) {
+          if (!mbar_wait(tile_req, rph, p.watch, kErrTimeoutProducer)) break;
+          rph ^= 1;
+        }
         // (no dynamic tiles when a stream-K tail deals them out statically)
         const int got = dp_tiles > 0 && sp.S == 0 ? atomicAdd(&p.sched[0], 1) : dp_tiles;
         const int T = got < dp_tiles ? got : -1;

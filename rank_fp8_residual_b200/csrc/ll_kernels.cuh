@@ -326,7 +326,6 @@ struct MainParams {
   int n_ftiles, n_ttiles;
   int lr_from_primary;  // 1: t is produced by the preceding kernel (wait on it)
   int withhold;         // debug: the TMA producer issues nothing
-  int act;              // epilogue activation (epi_act)
   Watch watch;
 };
 
@@ -344,6 +343,7 @@ __host__ __device__ constexpr int main_smem_bytes() {
   return kSX * kXSlot + kSQ * kQSlot + kEpiBytes + 1024 /*align*/ + 512 /*barriers*/;
 }
 
+template <int kAct>
 __global__ void __launch_bounds__(kMainThreads, 1) ll_main_kernel(const __grid_constant__ MainParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(kMainThreads, 1) ll_main_kernel(const __grid_c
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float v = fmaf(s, __uint_as_float(aq[i]), __uint_as_float(al[i]) + b);
-          st[i * 32 + lane] = to_bf16_bits(epi_act(v, p.act));
+          st[i * 32 + lane] = to_bf16_bits(epi_act<kAct>(v));
         }
         fence_proxy_async_smem();
         __syncwarp();

@@ -59,7 +59,6 @@ struct StreamParams {
   int dims3;             // 1: one 3-D load per group of 4 chunks; 0: four 2-D loads
   int lr_from_primary;   // 1: t is produced by the preceding kernel
   int withhold;          // debug: the TMA producers issue nothing
-  int act;               // epilogue activation (epi_act)
   Watch watch;
 };
 
@@ -87,6 +86,7 @@ __host__ __device__ constexpr int st_smem_bytes(int Mt) {
 }
 __host__ __device__ constexpr int st_smem_max() { return st_smem_bytes(kStMaxMt); }
 
+template <int kAct>
 __global__ void __launch_bounds__(kStThreads, 1) ll_stream_kernel(const __grid_constant__ StreamParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kStThreads, 1) ll_stream_kernel(const __grid_c
           for (int i = 0; i < 16; ++i) {
             const int m = cb + i;
             const float lr = has_lr ? __uint_as_float(al[i]) : 0.f;
-            if (m < p.M) p.y[static_cast<size_t>(m) * p.N + f] = to_bf16_bits(epi_act(fmaf(sc, __uint_as_float(aq[i]), lr + b), p.act));
+            if (m < p.M) p.y[static_cast<size_t>(m) * p.N + f] = to_bf16_bits(epi_act<kAct>(fmaf(sc, __uint_as_float(aq[i]), lr + b)));
           }
         }
       }

@@ -63,7 +63,6 @@ struct TcParams {
   int q3;                // 1: one 3-D Q load per stage; 0: two 2-D loads
   int lr_from_primary;
   int withhold;
-  int act;               // epilogue activation (epi_act)
   Watch watch;
 };
 
@@ -99,6 +98,7 @@ __device__ __forceinline__ void tc_tile_coords(int T, int n_ftiles, int n_ttiles
   t0 = (first_tt + idx % gsize) * bt;
 }
 
+template <int kAct>
 __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ll_tc_kernel(const __grid_const
         __syncwarp();
         uint16_t* st = stage + eb * (32 * 32);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) st[i * 32 + lane] = to_bf16_bits(epi_act(fmaf(s, __uint_as_float(v[i]), b), p.act));
+        for (int i = 0; i < 32; ++i) st[i * 32 + lane] = to_bf16_bits(epi_act<kAct>(fmaf(s, __uint_as_float(v[i]), b)));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

@@ -65,7 +65,6 @@ struct Tc2Params {
   int* sched;    // [2]: tile counter, finished-leader counter (0 between launches)
   int lr_from_primary;
   int withhold;
-  int act;       // epilogue activation (epi_act)
   Watch watch;
 };
 
@@ -128,6 +127,7 @@ struct TileRing {
   }
 };
 
+template <int kAct>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
     ll_tc2_kernel(const __grid_constant__ Tc2Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -464,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
         __syncwarp();
         uint16_t* st = stage + eb * (32 * 32);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) st[i * 32 + lane] = to_bf16_bits(epi_act(fmaf(s, __uint_as_float(v[i]), b), p.act));
+        for (int i = 0; i < 32; ++i) st[i * 32 + lane] = to_bf16_bits(epi_act<kAct>(fmaf(s, __uint_as_float(v[i]), b)));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

@@ -489,7 +489,16 @@ __device__ __forceinline__ float gelu_tanh(float v) {
   const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
   return 0.5f * v * (1.f + tanhf(u));
 }
-__device__ __forceinline__ float epi_act(float v, int act) { return act == 1 ? gelu_tanh(v) : v; }
+// Epilogue activation, fixed at compile time so that the identity
+// instantiation carries none of the activation's code or registers.
+constexpr int kActNone = 0, kActGelu = 1, kActGeglu = 2;
+template <int kAct>
+__device__ __forceinline__ float epi_act(float v) {
+  if constexpr (kAct == kActGelu)
+    return gelu_tanh(v);
+  else
+    return v;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
