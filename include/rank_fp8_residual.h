@@ -65,16 +65,19 @@ enum {
 };
 
 /* Kernel variants for ll_set_variant (no counterpart on the pages).  AUTO:
- * STREAM for M <= 64, TC_PAIR for 64 < M <= 256, TC above (the measured
- * crossovers).  TC: one-CTA fused
+ * STREAM for M <= 64, TC_PAIR for 64 < M <= 256, above TC or FP8_SPLIT
+ * (FP8_SPLIT on wide layers: N >= 2K, or N >= K at M >= 4096; the
+ * measured crossovers).  TC: one-CTA fused
  * kernel, 128 features x up to 256 tokens per tile, low-rank factor folded
  * as A / scale (bf16 pair).  TC_PAIR: the same on CTA pairs (256 features
  * per MMA, tiles as narrow as 32 tokens).  SMALL: one-CTA
  * kernel, 128 x 128 tiles, separate residual and low-rank accumulators.
  * STREAM (M <= 64 only; larger M runs SMALL): one CTA per 128 features
  * streaming Q in 32 KB boxes, all tokens in one MMA, exact A.  FP8_SPLIT:
- * CTA pairs on e4m3 tensor cores (kind::f8f6f4) with Q as stored and x
- * carried per token as the two-term e4m3fn expansion of ll_quantize_x.
+ * e4m3 tensor cores (kind::f8f6f4) with Q as stored and x carried per
+ * token as the two-term e4m3fn expansion of ll_quantize_x: CTA pairs on
+ * 256 x 256 tiles above 64 tokens; up to 64 tokens (except with the GEGLU
+ * epilogue) a streaming kernel that deals Q's bytes out evenly to the SMs.
  * These variants meet the same accuracy bound.  FP8_ACT: the same kernel
  * on one e4m3fn term per token, the FP8-activation variant: its result is
  * the layer's formula evaluated on x quantised per token as by

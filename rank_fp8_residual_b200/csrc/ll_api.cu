@@ -20,6 +20,7 @@
 #include "ll_tc2.cuh"
 #include "ll_stream.cuh"
 #include "ll_f8.cuh"
+#include "ll_f8_stream.cuh"
 #include "ll_decompose.cuh"
 
 namespace {
@@ -164,6 +165,7 @@ struct CallMaps {
   CUtensorMap c_x2p, c_thip, c_tlop;  // CTA-pair kernel: x and t boxes of bt2 / 2 rows
   int c_bt2 = 0;
   CUtensorMap c_xh, c_xl, c_thi32, c_tlo32, c_y64;  // FP8-operand kernel
+  CUtensorMap c_xhs, c_xls;                         // FP8-operand streaming kernel: code boxes of Mt rows
 };
 constexpr int kMapCache = 8;  // descriptor sets kept per layer (e.g. the chunks of a host-buffer forward)
 
@@ -278,6 +280,10 @@ Tc2Fn kernel_tc2(int act) { return act == llk::kActGelu ? llk::ll_tc2_kernel<llk
 StreamFn kernel_stream(int act) {
   return act == llk::kActGelu ? llk::ll_stream_kernel<llk::kActGelu> : llk::ll_stream_kernel<llk::kActNone>;
 }
+using F8sFn = void (*)(llk::F8sParams);
+F8sFn kernel_f8s(int act) {
+  return act == llk::kActGelu ? llk::ll_f8_stream_kernel<llk::kActGelu> : llk::ll_f8_stream_kernel<llk::kActNone>;
+}
 F8Fn kernel_f8(int act) {
   return act == llk::kActGeglu  ? llk::ll_f8_kernel<llk::kActGeglu>
          : act == llk::kActGelu ? llk::ll_f8_kernel<llk::kActGelu>
@@ -299,6 +305,7 @@ int set_smem_attrs_once() {
       smem(kernel_tc(a), llk::tc_smem_bytes());
       smem(kernel_tc2(a), llk::tc2_smem_bytes());
       smem(kernel_stream(a), llk::st_smem_max());
+      smem(kernel_f8s(a), llk::ss_smem_max());
     }
     for (int a = 0; a < 3; ++a) smem(kernel_f8(a), llk::f8_smem_bytes());
     smem(llk::ll_lrdown_kernel, llk::lr_smem_bytes(256));
@@ -383,7 +390,7 @@ int ensure_f8_workspace(ll_layer* h, int M, cudaStream_t st) {
   return LL_OK;
 }
 
-enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM, PATH_F8 };
+enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM, PATH_F8, PATH_F8S };
 
 bool is_geglu(const ll_layer* h) { return h->epilogue == LL_EPILOGUE_GEGLU_TANH; }
 // Columns of y: N, or N / 2 when the epilogue is GEGLU.
@@ -406,10 +413,15 @@ int act_code(const ll_layer* h) {
 bool fp8_split_wins(int N, int K, int M) { return N >= 2 * K || (N >= K && M >= 4096); }
 
 constexpr int kStreamMaxM = 64;
+constexpr int kF8sLrBudget = 20;  // SMs for the down-projection beside the FP8-operand streaming kernel
 constexpr int kPairMaxM = 256;
 
 Path choose_path(const ll_layer* h, int M) {
-  if (h->variant == LL_VARIANT_FP8_SPLIT || h->variant == LL_VARIANT_FP8_ACT) return PATH_F8;
+  // The FP8-operand variants: the streaming kernel up to 64 tokens (not with
+  // GEGLU, whose value and gate rows sit in different 128-feature tiles
+  // there), the CTA-pair kernel above.
+  if (h->variant == LL_VARIANT_FP8_SPLIT || h->variant == LL_VARIANT_FP8_ACT)
+    return M <= kStreamMaxM && !is_geglu(h) ? PATH_F8S : PATH_F8;
   // GEGLU pairs value and gate features inside a thread: the FP8-operand
   // kernel holds a token's features in one thread; the others do not.
   if (is_geglu(h) && h->variant == LL_VARIANT_AUTO) return PATH_F8;
@@ -563,6 +575,9 @@ LrPlan plan_lowrank(const ll_layer* h, int M) {
   // Beside the FP8-operand kernel, whose tiles need t only at their end:
   // half of the SMs.
   if (path == PATH_F8) budget = std::max(1, h->num_sms / 2);
+  // Beside the FP8-operand streaming kernel: about as many SMs as the
+  // exact streaming kernel leaves free at the small-batch shape.
+  if (path == PATH_F8S) budget = kF8sLrBudget;
   int ks = std::max(1, budget / ctas);
   ks = std::min(std::min(ks, nK), llk::kLrMaxSplit);
   if (path == PATH_TC1 && M > 128) ks = plan_tc1(h, M).ks;
@@ -626,6 +641,11 @@ bool build_call_maps_uncached(ll_layer* h, const void* x, void* y, int M, bool f
     ok &= make_map(&h->cm.c_xl, h->xl, kU8, M, h->K, h->K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&h->cm.c_y64, y, kBF16, M, out_features(h), 2ull * out_features(h), 32, 32,
                    CU_TENSOR_MAP_SWIZZLE_64B);
+    if (M <= kStreamMaxM) {
+      const uint32_t Mt = static_cast<uint32_t>((M + 15) / 16 * 16);
+      ok &= make_map(&h->cm.c_xhs, h->xh, kU8, M, h->K, h->K, 128, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&h->cm.c_xls, h->xl, kU8, M, h->K, h->K, 128, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     if (h->r_pad > 0) {
       ok &= make_map(&h->cm.c_thi32, h->t_hi, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
       ok &= make_map(&h->cm.c_tlo32, h->t_lo, kBF16, M, h->r_pad, 2ull * h->r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -745,14 +765,15 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   h->last_launches = 0;
   const Path path = choose_path(h, M);
   if (is_geglu(h) && path != PATH_F8) return LL_ERR_UNSUPPORTED;
+  const bool f8 = path == PATH_F8 || path == PATH_F8S;
   const LrPlan lp = plan_lowrank(h, M);
   int rc = ensure_workspace(h, M, st);
   if (rc != LL_OK) return rc;
-  if (path == PATH_F8) {
+  if (f8) {
     rc = ensure_f8_workspace(h, M, st);
     if (rc != LL_OK) return rc;
   }
-  if (!build_call_maps(h, x, y, M, path == PATH_F8)) return LL_ERR_CUDA;
+  if (!build_call_maps(h, x, y, M, f8)) return LL_ERR_CUDA;
   const Watch watch{h->status, h->timeout_ns};
   int launches = 0;
   const bool prof = h->profiling != 0;
@@ -764,7 +785,7 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
   }
 
   const int f8_terms = h->variant == LL_VARIANT_FP8_ACT ? 1 : 2;
-  if (path == PATH_F8) {
+  if (f8) {
     // Per-token exponents and e4m3 codes of x; the down-projection and the
     // FP8-operand kernel below both read them.
     const int blocks = std::max(1, std::min((M + 7) / 8, h->num_sms * 8));
@@ -793,9 +814,9 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     lpp.tmem_cols = lp.tmem_cols;
     lpp.ksplit = lp.ksplit;
     lpp.kb_per_split = lp.kb_per_split;
-    lpp.e_tok = path == PATH_F8 ? h->e_tok : nullptr;
+    lpp.e_tok = f8 ? h->e_tok : nullptr;
     // Beside the split of x, which writes the token exponents it reads.
-    lpp.wait_prior = path == PATH_F8 && !prof ? 1 : 0;
+    lpp.wait_prior = f8 && !prof ? 1 : 0;
     lpp.watch = watch;
     const cudaError_t lerr = launch_lrdown(lpp, lp, st);
     h->names[launches++] = "ll_lrdown_kernel";
@@ -860,6 +881,41 @@ int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) 
     cfg.dynamicSmemBytes = f8_smem_bytes();
     err = cudaLaunchKernelEx(&cfg, kernel_f8(act_code(h)), fp);
     h->names[launches] = "ll_f8_kernel";
+  } else if (path == PATH_F8S) {
+    F8sParams fs;
+    fs.tm_q = h->tm_q128;
+    fs.tm_xh = h->cm.c_xhs;
+    fs.tm_xl = h->cm.c_xls;
+    fs.tm_a = h->r_pad > 0 ? h->tm_a : h->tm_q128;  // unused when r_pad == 0
+    fs.tm_thi = h->r_pad > 0 ? h->cm.c_this : h->cm.c_xhs;
+    fs.tm_tlo = h->r_pad > 0 ? h->cm.c_tlos : h->cm.c_xhs;
+    fs.e_tok = h->e_tok;
+    fs.scale = h->scale;
+    fs.bias = h->has_bias ? h->bias : nullptr;
+    fs.y = static_cast<uint16_t*>(y);
+    fs.part = h->f8_part;
+    fs.cnt = h->f8_cnt;
+    fs.M = M;
+    fs.N = h->N;
+    fs.K = h->K;
+    fs.r_pad = h->r_pad;
+    fs.Mt = (M + 15) / 16 * 16;
+    fs.terms = f8_terms;
+    fs.n_ftiles = (h->N + 127) / 128;
+    // One CTA per SM that the down-projection leaves free; at most one per unit.
+    const int lr_ctas = h->r_pad > 0 ? lp.m_tiles * lp.r_chunks * lp.ksplit : 0;
+    const long long units =
+        static_cast<long long>(fs.n_ftiles) * ((h->K + 127) / 128 + (h->r_pad + 63) / 64);
+    fs.ctas = static_cast<int>(std::max(1LL, std::min<long long>(std::max(1, h->num_sms - lr_ctas), units)));
+    fs.w_stages = ss_w_stages(fs.Mt);
+    fs.lr_from_primary = overlap ? 1 : 0;
+    fs.withhold = h->withhold;
+    fs.watch = watch;
+    cfg.gridDim = dim3(fs.ctas);
+    cfg.blockDim = dim3(kSsThreads);
+    cfg.dynamicSmemBytes = ss_smem_bytes(fs.Mt);
+    err = cudaLaunchKernelEx(&cfg, kernel_f8s(act_code(h)), fs);
+    h->names[launches] = "ll_f8_stream_kernel";
   } else if (path == PATH_STREAM) {
     StreamParams sp;
     const bool dims3 = h->K % 64 == 0;
@@ -1376,6 +1432,10 @@ int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int* kernel, i
     case PATH_F8:
       kv = variant == LL_VARIANT_FP8_ACT ? LL_VARIANT_FP8_ACT : LL_VARIANT_FP8_SPLIT;
       bt = 256;
+      break;
+    case PATH_F8S:
+      kv = variant == LL_VARIANT_FP8_ACT ? LL_VARIANT_FP8_ACT : LL_VARIANT_FP8_SPLIT;
+      bt = (M + 15) / 16 * 16;
       break;
     case PATH_SMALL:
       break;
