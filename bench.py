@@ -104,6 +104,9 @@ KERNEL_SOURCES = {
     "ll_stream_kernel": ["ll_stream.cuh", "ll_kernels.cuh", "ptx.cuh"],
     "ll_f8_kernel": ["ll_f8.cuh", "ll_kernels.cuh", "ptx.cuh"],
     "ll_xsplit_kernel": ["ll_f8.cuh", "ll_kernels.cuh", "ptx.cuh"],
+    "ll_f8_stream_kernel": ["ll_f8_stream.cuh", "ll_kernels.cuh", "ptx.cuh"],
+    "ll_gemv_kernel": ["ll_gemv.cuh", "ll_kernels.cuh", "ptx.cuh"],
+    "ll_gemv_t_kernel": ["ll_gemv.cuh", "ll_kernels.cuh", "ptx.cuh"],
 }
 
 
@@ -262,7 +265,7 @@ def run_reference(args, w):
     return 0
 
 
-VARIANT_NAMES = ("auto", "tc", "tc_pair", "small", "stream", "fp8_split", "fp8_act")
+VARIANT_NAMES = ("auto", "tc", "tc_pair", "small", "stream", "fp8_split", "fp8_act", "gemv")
 
 
 def variant_id(ll, name):

@@ -65,7 +65,8 @@ enum {
 };
 
 /* Kernel variants for ll_set_variant (no counterpart on the pages).  AUTO:
- * STREAM for M <= 64, TC_PAIR for 64 < M <= 256, above TC or FP8_SPLIT
+ * GEMV for M == 1 (when x fits), STREAM for M <= 64, TC_PAIR for
+ * 64 < M <= 256, above TC or FP8_SPLIT
  * (FP8_SPLIT on wide layers: N >= 2K, or N >= K at M >= 4096; the
  * measured crossovers).  TC: one-CTA fused
  * kernel, 128 features x up to 256 tokens per tile, low-rank factor folded
@@ -82,7 +83,10 @@ enum {
  * on one e4m3fn term per token, the FP8-activation variant: its result is
  * the layer's formula evaluated on x quantised per token as by
  * ll_quantize_x with terms == 1 (that rounding of x is part of the
- * variant's definition). */
+ * variant's definition).  GEMV (M <= 4 with x in shared memory beside the
+ * 128 KB load ring, 2*M*K + 128 KB + 128 bytes <= 227 KB; otherwise SMALL):
+ * CUDA cores only, every weight element used by M fused multiply-adds and
+ * warp reductions, t in fp32; it meets the same accuracy bound. */
 enum {
   LL_VARIANT_AUTO = 0,
   LL_VARIANT_TC = 1,
@@ -90,7 +94,8 @@ enum {
   LL_VARIANT_TC_PAIR = 3,
   LL_VARIANT_STREAM = 4,
   LL_VARIANT_FP8_SPLIT = 5,
-  LL_VARIANT_FP8_ACT = 6
+  LL_VARIANT_FP8_ACT = 6,
+  LL_VARIANT_GEMV = 7
 };
 
 /* LiteLinear README, "Usage": the layer constructor

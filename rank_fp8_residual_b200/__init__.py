@@ -37,6 +37,7 @@ LL_VARIANT_TC_PAIR = 3
 LL_VARIANT_STREAM = 4
 LL_VARIANT_FP8_SPLIT = 5
 LL_VARIANT_FP8_ACT = 6
+LL_VARIANT_GEMV = 7
 
 LL_EPILOGUE_NONE = 0
 LL_EPILOGUE_GELU_TANH = 1

@@ -21,6 +21,7 @@
 #include "ll_stream.cuh"
 #include "ll_f8.cuh"
 #include "ll_f8_stream.cuh"
+#include "ll_gemv.cuh"
 #include "ll_decompose.cuh"
 
 namespace {
@@ -199,6 +200,7 @@ struct ll_layer {
   int* f8_cnt = nullptr;     // arrival counters of K-split tiles, [tiles of ws8_M rows][2][4]
   size_t f8_cnt_n = 0;
   float* f8_part = nullptr;  // fp32 partial tiles, two slots per CTA pair
+  float* t32 = nullptr;      // GEMV path: t in fp32, [kGvMaxM, r_pad]
   CUtensorMap tm_q128, tm_ahi32, tm_alo32;     // set-time maps of the FP8-operand kernel
   mutable int f8_clusters = 0;                 // co-resident clusters of the FP8-operand kernel
   // host-buffer forward staging: device copies of x and y, and two copy
@@ -265,6 +267,7 @@ void free_layer_mem(ll_layer* h) {
   cudaFree(h->xl);
   cudaFree(h->f8_cnt);
   cudaFree(h->f8_part);
+  cudaFree(h->t32);
 }
 
 // The epilogue activation is a template parameter of each kernel (see
@@ -290,6 +293,29 @@ F8Fn kernel_f8(int act) {
                                 : llk::ll_f8_kernel<llk::kActNone>;
 }
 
+using GemvTFn = void (*)(const uint16_t*, const uint16_t*, float*, int, int);
+using GemvFn = void (*)(llk::GemvParams);
+template <int kM>
+GemvFn gemv_kernel_m(int act) {
+  return act == llk::kActGelu ? llk::ll_gemv_kernel<kM, llk::kActGelu> : llk::ll_gemv_kernel<kM, llk::kActNone>;
+}
+GemvFn kernel_gemv(int M, int act) {
+  switch (M) {
+    case 1: return gemv_kernel_m<1>(act);
+    case 2: return gemv_kernel_m<2>(act);
+    case 3: return gemv_kernel_m<3>(act);
+    default: return gemv_kernel_m<4>(act);
+  }
+}
+GemvTFn kernel_gemv_t(int M) {
+  switch (M) {
+    case 1: return llk::ll_gemv_t_kernel<1>;
+    case 2: return llk::ll_gemv_t_kernel<2>;
+    case 3: return llk::ll_gemv_t_kernel<3>;
+    default: return llk::ll_gemv_t_kernel<4>;
+  }
+}
+
 int set_smem_attrs_once() {
   static int rc = -1;
   static std::once_flag once;
@@ -308,6 +334,19 @@ int set_smem_attrs_once() {
       smem(kernel_f8s(a), llk::ss_smem_max());
     }
     for (int a = 0; a < 3; ++a) smem(kernel_f8(a), llk::f8_smem_bytes());
+    // The GEMV pair shares SMs while the t kernel runs: both ask for the
+    // largest shared-memory carve-out, so an SM need not be reconfigured.
+    auto carve = [](auto f) {
+      if (cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) rc = 1;
+    };
+    for (int m = 1; m <= llk::kGvMaxM; ++m) {
+      smem(kernel_gemv_t(m), 227 * 1024 - llk::kGvRingBytes);
+      carve(kernel_gemv_t(m));
+      for (int a = 0; a < 2; ++a) {
+        smem(kernel_gemv(m, a), 227 * 1024);
+        carve(kernel_gemv(m, a));
+      }
+    }
     smem(llk::ll_lrdown_kernel, llk::lr_smem_bytes(256));
   });
   return rc;
@@ -390,7 +429,7 @@ int ensure_f8_workspace(ll_layer* h, int M, cudaStream_t st) {
   return LL_OK;
 }
 
-enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM, PATH_F8, PATH_F8S };
+enum Path { PATH_SMALL, PATH_TC1, PATH_TC2, PATH_STREAM, PATH_F8, PATH_F8S, PATH_GEMV };
 
 bool is_geglu(const ll_layer* h) { return h->epilogue == LL_EPILOGUE_GEGLU_TANH; }
 // Columns of y: N, or N / 2 when the epilogue is GEGLU.
@@ -413,6 +452,9 @@ int act_code(const ll_layer* h) {
 bool fp8_split_wins(int N, int K, int M) { return N >= 2 * K || (N >= K && M >= 4096); }
 
 constexpr int kStreamMaxM = 64;
+bool gemv_fits(const ll_layer* h, int M) {
+  return M <= llk::kGvMaxM && llk::gv_smem_bytes(M, h->K) <= 227u * 1024u;
+}
 constexpr int kF8sLrBudget = 20;  // SMs for the down-projection beside the FP8-operand streaming kernel
 constexpr int kPairMaxM = 256;
 
@@ -425,10 +467,16 @@ Path choose_path(const ll_layer* h, int M) {
   // GEGLU pairs value and gate features inside a thread: the FP8-operand
   // kernel holds a token's features in one thread; the others do not.
   if (is_geglu(h) && h->variant == LL_VARIANT_AUTO) return PATH_F8;
+  // CUDA-core GEMV: M <= 4 with x fitting in shared memory beside the ring.
+  if (h->variant == LL_VARIANT_GEMV) return gemv_fits(h, M) ? PATH_GEMV : PATH_SMALL;
   if (h->variant == LL_VARIANT_TC) return PATH_TC1;
   if (h->variant == LL_VARIANT_TC_PAIR) return PATH_TC2;
   if (h->variant == LL_VARIANT_SMALL) return PATH_SMALL;
   if (h->variant == LL_VARIANT_STREAM) return M <= kStreamMaxM ? PATH_STREAM : PATH_SMALL;
+  // One token: the CUDA-core GEMV (measured at K = 4096, N = 16384,
+  // r = 512: 29.7 against 31.8 us; from two tokens on the streaming kernel
+  // leads, 31.7 against 33.8).
+  if (M == 1 && gemv_fits(h, M)) return PATH_GEMV;
   if (M <= kStreamMaxM) return PATH_STREAM;
   // Measured on the K = 4096, N = 16384 family: the CTA-pair kernel with
   // its narrow tiles beats the 128 x 128 and one-CTA kernels up to 256
@@ -760,11 +808,76 @@ int pair_cluster_count(const ll_layer* h) {
   return h->pair_clusters;
 }
 
+// M <= 4 on CUDA cores: t = x B^T (fp32) and the fused GEMV, a programmatic
+// dependent of it that waits only before its low-rank part.
+int forward_gemv(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) {
+  using namespace llk;
+  if (h->r_pad > 0 && !h->t32) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&h->t32), sizeof(float) * kGvMaxM * h->r_pad, st) != cudaSuccess) {
+      cudaGetLastError();
+      h->t32 = nullptr;
+      return LL_ERR_OOM;
+    }
+  }
+  int launches = 0;
+  const bool prof = h->profiling != 0;
+  h->prof_valid = 0;
+  if (prof) {
+    for (cudaEvent_t& e : h->ev)
+      if (!e && cudaEventCreate(&e) != cudaSuccess) return LL_ERR_CUDA;
+    cudaEventRecord(h->ev[0], st);
+  }
+  if (h->r_pad > 0) {
+    const int grid = std::max(1, std::min(h->num_sms, (h->r_pad + kGvWarps - 1) / kGvWarps));
+    kernel_gemv_t(M)<<<grid, kGvThreads, static_cast<size_t>(M) * h->K * 2, st>>>(
+        static_cast<const uint16_t*>(x), h->B, h->t32, h->K, h->r_pad);
+    h->names[launches++] = "ll_gemv_t_kernel";
+    if (prof) cudaEventRecord(h->ev[launches], st);
+    if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
+  }
+  GemvParams gp;
+  gp.x = static_cast<const uint16_t*>(x);
+  gp.q = h->Q;
+  gp.a = h->A;
+  gp.t = h->t32;
+  gp.scale = h->scale;
+  gp.bias = h->has_bias ? h->bias : nullptr;
+  gp.y = static_cast<uint16_t*>(y);
+  gp.M = M;
+  gp.N = h->N;
+  gp.K = h->K;
+  gp.r_pad = h->r_pad;
+  const bool overlap = h->r_pad > 0 && !prof;
+  gp.t_from_primary = overlap ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = st;
+  cfg.gridDim = dim3(h->num_sms);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = gv_smem_bytes(M, h->K);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kernel_gemv(M, act_code(h)), gp) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
+  h->names[launches++] = "ll_gemv_kernel";
+  if (prof) {
+    cudaEventRecord(h->ev[launches], st);
+    h->prof_valid = 1;
+  }
+  h->last_launches = launches;
+  return LL_OK;
+}
+
 int forward_device(ll_layer* h, const void* x, void* y, int M, cudaStream_t st) {
   using namespace llk;
   h->last_launches = 0;
   const Path path = choose_path(h, M);
   if (is_geglu(h) && path != PATH_F8) return LL_ERR_UNSUPPORTED;
+  if (path == PATH_GEMV) return forward_gemv(h, x, y, M, st);
   const bool f8 = path == PATH_F8 || path == PATH_F8S;
   const LrPlan lp = plan_lowrank(h, M);
   int rc = ensure_workspace(h, M, st);
@@ -1392,7 +1505,7 @@ int ll_set_epilogue(ll_handle h, int epilogue) {
 
 int ll_set_variant(ll_handle h, int variant) {
   g_last_error = LL_OK;
-  if (!h || (variant < LL_VARIANT_AUTO || variant > LL_VARIANT_FP8_ACT))
+  if (!h || (variant < LL_VARIANT_AUTO || variant > LL_VARIANT_GEMV))
     return fail(LL_ERR_INVALID_ARG);
   h->variant = variant;
   return LL_OK;
@@ -1401,7 +1514,7 @@ int ll_set_variant(ll_handle h, int variant) {
 int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int* kernel, int* tile_tokens, int* lr_splits) {
   g_last_error = LL_OK;
   if (N < 1 || K < 16 || r < 0 || (N % 8) != 0 || (K % 16) != 0 || M < 1 || num_sms < 2 ||
-      (variant < LL_VARIANT_AUTO || variant > LL_VARIANT_FP8_ACT))
+      (variant < LL_VARIANT_AUTO || variant > LL_VARIANT_GEMV))
     return fail(LL_ERR_INVALID_ARG);
   if (r > 512) return fail(LL_ERR_UNSUPPORTED);
   // A handle-shaped view holding only what the planning reads.
@@ -1437,12 +1550,16 @@ int ll_plan(int N, int K, int r, int M, int num_sms, int variant, int* kernel, i
       kv = variant == LL_VARIANT_FP8_ACT ? LL_VARIANT_FP8_ACT : LL_VARIANT_FP8_SPLIT;
       bt = (M + 15) / 16 * 16;
       break;
+    case PATH_GEMV:
+      kv = LL_VARIANT_GEMV;
+      bt = M;
+      break;
     case PATH_SMALL:
       break;
   }
   if (kernel) *kernel = kv;
   if (tile_tokens) *tile_tokens = bt;
-  if (lr_splits) *lr_splits = view.r_pad > 0 ? plan_lowrank(&view, M).ksplit : 1;
+  if (lr_splits) *lr_splits = view.r_pad > 0 && path != PATH_GEMV ? plan_lowrank(&view, M).ksplit : 1;
   return LL_OK;
 }
 

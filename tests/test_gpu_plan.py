@@ -9,10 +9,10 @@ pytestmark = pytest.mark.gpu
 
 NAMES = {ll.LL_VARIANT_TC: "ll_tc_kernel", ll.LL_VARIANT_TC_PAIR: "ll_tc2_kernel",
          ll.LL_VARIANT_SMALL: "ll_main_kernel", ll.LL_VARIANT_STREAM: "ll_stream_kernel",
-         ll.LL_VARIANT_FP8_SPLIT: "ll_f8_kernel"}
+         ll.LL_VARIANT_FP8_SPLIT: "ll_f8_kernel", ll.LL_VARIANT_GEMV: "ll_gemv_kernel"}
 
 
-@pytest.mark.parametrize("M,N", [(16, 2048), (64, 2048), (100, 2048), (256, 2048), (300, 2048), (1024, 2048),
+@pytest.mark.parametrize("M,N", [(1, 2048), (16, 2048), (64, 2048), (100, 2048), (256, 2048), (300, 2048), (1024, 2048),
                                  (300, 4096), (1024, 4096)])
 def test_plan_matches_launched_kernel(M, N):
     K, r = 1024, 64
@@ -32,6 +32,8 @@ def test_plan_matches_launched_kernel(M, N):
         assert names[-1] == NAMES[kernel]
         if kernel == ll.LL_VARIANT_FP8_SPLIT:
             assert names[:2] == ["ll_xsplit_kernel", "ll_lrdown_kernel"]
+        elif kernel == ll.LL_VARIANT_GEMV:
+            assert names[0] == "ll_gemv_t_kernel"
         else:
             assert names[0] == "ll_lrdown_kernel"
     finally:
