@@ -127,3 +127,17 @@ def test_misaligned_pointers_are_rejected_before_any_gpu_work():
         with pytest.raises(ll.LLError) as e:
             ll.ll_quantize_x(x, 8, 64, 2, e_out, hi, lo, stream=0)
         assert e.value.code == ll.LL_ERR_INVALID_ARG
+
+
+def test_binding_constants_match_the_header():
+    """Every `LL_NAME = value` enumerator of include/*.h has the same value in
+    the Python binding."""
+    import rank_fp8_residual_b200 as ll
+    found = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for name, val in re.findall(r"\b(LL_[A-Z_0-9]+)\s*=\s*(\d+)", src):
+            found[name] = int(val)
+    assert "LL_VARIANT_GEMV" in found and "LL_EPILOGUE_GEGLU_TANH" in found
+    for name, val in found.items():
+        assert getattr(ll, name) == val, name
